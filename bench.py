@@ -1,0 +1,420 @@
+"""Benchmark of the tile-sparse attention layer (TripPool -> projection/score ->
+Top-k -> tile-skipping attention) on the 245,760-token long-video workload
+(B=1, H=32, d=128, grid 60x64x64, head-aware 128-token tiles, 1,920 tiles,
+k=96 = 95% sparsity).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {veda,reference}]
+
+A step is one pass of the whole layer over one batch of synthetic input.  The
+timed region covers K steps on the device (CUDA events, barrier + synchronize
+on both sides, max over ranks).  Inputs (Q/K/V 6 GB) are larger than L2.  The
+metric is ms/layer and effective TFLOP/s: the FLOPs of the selected tile pairs
+only (4 * B*H*nT*k*Bt^2*d = 4.948e13), mask preparation included in the time.
+
+Multi-GPU: every rank runs its own layer (independent batch entries, no
+data-path collective): weak scaling; value = FLOPs of all ranks / max time.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload (the reference arm; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "ms/layer and effective TFLOP/s of tile-sparse attention (+mask prep) at 95% sparsity"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- distributed
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[3][1:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w, t_host, heads=1, units_per_head=24, threads=None):
+    """Times the fp64 oracle on a bounded sample of the layer and extrapolates.
+
+    Sample: full mask preparation for ``heads`` heads (TripPool, projection,
+    score, Top-k) and attention for ``units_per_head`` query tiles of each.
+    Heads and query tiles are independent units of equal cost, so the full
+    layer time is linear in them.
+    """
+    from oracle import Oracle
+    o = Oracle()
+    if threads:
+        o.set_num_threads(threads)
+    hs = list(range(heads))
+    Qb = np.ascontiguousarray(t_host["Q"][:, hs])
+    Kb = np.ascontiguousarray(t_host["K"][:, hs])
+    Vb = np.ascontiguousarray(t_host["V"][:, hs])
+    shapes = [w.tile_shapes[h] for h in hs]
+    t0 = time.perf_counter()
+    r = o.mask_prep(Qb, Kb, t_host["Wq"][hs], t_host["Wk"][hs], w.grid, shapes, w.k)
+    t1 = time.perf_counter()
+    rng = np.random.default_rng(0)
+    units = np.array([(0, h, int(i)) for h in range(heads)
+                      for i in rng.choice(w.nT, units_per_head, replace=False)], dtype=np.int64)
+    o.sparse_attention(Qb, Kb, Vb, r["idx"], w.grid, shapes, w.scale, units=units)
+    t2 = time.perf_counter()
+    prep_per_head = (t1 - t0) / heads
+    attn_per_unit = (t2 - t1) / len(units)
+    full_s = prep_per_head * w.B * w.H + attn_per_unit * w.B * w.H * w.nT
+    return dict(seconds_sampled=t2 - t0, full_layer_s=full_s, cores=o.num_threads(),
+                sample=f"mask prep of {heads} head(s) + attention of {len(units)} query tiles "
+                       f"of {w.name}; full layer extrapolated linearly over heads and query tiles")
+
+
+def host_inputs(w, t):
+    return {"Q": workloads.bf16_bits(t["Q"]), "K": workloads.bf16_bits(t["K"]),
+            "V": workloads.bf16_bits(t["V"]), "Wq": t["Wq"].cpu().numpy(),
+            "Wk": t["Wk"].cpu().numpy()}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return 0
+    # inputs drawn on the CPU: only the sampled heads are needed
+    wh = workloads.Workload(w.name, w.B, 1, w.d, w.T, w.Hs, w.Ws, w.tile_shapes[:1], w.k,
+                            w.sparsity, w.seed)
+    t = workloads.generate(wh, device="cpu")
+    th = host_inputs(wh, t)
+    times = []
+    res = None
+    for s in range(args.warmup + args.steps):
+        res = oracle_sample(w, th, heads=1, units_per_head=8)
+        if s >= args.warmup:
+            times.append(res["full_layer_s"])
+    ms = 1e3 * statistics.mean(times)
+    value = w.sparse_flops() / (ms * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(w.describe(), parallelism="replicas"),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"],
+                             "kind": "oracle", "sample": res["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- main arm
+def run_veda(args, w, world, rank, local):
+    import tile_sparse_attention_b200 as vb
+    vb.load_library()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = _peaks()
+    t = workloads.generate(w, device=dev)
+    prob = vb.Problem.from_workload(w)
+    B, H, N, d, nT, k = w.B, w.H, w.N, w.d, w.nT, w.k
+    statsQ = torch.empty((B, H, nT, 3, d), dtype=torch.float32, device=dev)
+    statsK = torch.empty_like(statsQ)
+    S = torch.empty((B, H, nT, nT), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, H, nT, k), dtype=torch.int32, device=dev)
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ws = vb.alloc_workspace(prob, dev)
+    stream = torch.cuda.current_stream(dev)
+    nk = 5  # kernels per launch group below: tripool, 2x projection + score, topk, attention
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        vb.veda_tripool(prob, t["Q"], t["K"], statsQ, statsK)
+        if ev is not None:
+            ev[1].record(stream)
+        vb.veda_tile_score(prob, statsQ, statsK, t["Wq"], t["Wk"], S, ws)
+        if ev is not None:
+            ev[2].record(stream)
+        vb.veda_topk_mask(prob, S, None, idx)
+        if ev is not None:
+            ev[3].record(stream)
+        vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O, lse, ws)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert vb.veda_get_status(ws) == 0, "device status after warm-up"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        _barrier(world)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        _barrier(world)
+    clocks = clk.summary()
+    status = vb.veda_get_status(ws)
+    total_ms = start.elapsed_time(stop)
+    total_ms = _max_over_ranks(total_ms, world)
+    ms = total_ms / args.steps
+    per = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+           for i, n in enumerate(["tripool", "tile_score", "topk", "sparse_attn"])}
+    flops = w.sparse_flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # mask-prep kernels as a fraction of HBM bandwidth (algorithmic bytes)
+    tri_bytes = 2 * B * H * N * d * 2 + 2 * B * H * nT * 3 * d * 4
+    stats_b = B * H * nT * 3 * d * 4
+    score_bytes = 2 * stats_b + 2 * H * d * d * 4 + 2 * stats_b + 2 * stats_b + B * H * nT * nT * 4
+    topk_bytes = B * H * nT * nT * 4 + B * H * nT * k * 4
+    attn_tf = flops / (per["sparse_attn"] * 1e-3) / 1e12
+    mask_prep = {
+        "tripool": {"ms": per["tripool"], "GB_s": tri_bytes / per["tripool"] / 1e6,
+                    "frac_hbm": tri_bytes / per["tripool"] / 1e6 / peaks["hbm"]},
+        "tile_score": {"ms": per["tile_score"], "GB_s": score_bytes / per["tile_score"] / 1e6,
+                       "frac_hbm": score_bytes / per["tile_score"] / 1e6 / peaks["hbm"],
+                       "fp32_TFLOP_s": 2 * B * H * (2 * 3 * nT * d * d + nT * nT * 3 * d)
+                       / (per["tile_score"] * 1e-3) / 1e12},
+        "topk": {"ms": per["topk"], "GB_s": topk_bytes / per["topk"] / 1e6,
+                 "frac_hbm": topk_bytes / per["topk"] / 1e6 / peaks["hbm"]},
+    }
+
+    # the build's own dense path (k = nT, no index list), outside the timed region
+    dense_ms = None
+    if not args.no_dense:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], None, O, lse, ws)
+        e0.record(stream)
+        vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], None, O, lse, ws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        dense_ms = e0.elapsed_time(e1)
+
+    # end to end through the public call with host buffers (pinned), every step:
+    # H2D of Q, K, V, Wq, Wk; veda_forward; D2H of O.
+    e2e = None
+    if not args.no_e2e:
+        hostQ = t["Q"].cpu().pin_memory()
+        hostK = t["K"].cpu().pin_memory()
+        hostV = t["V"].cpu().pin_memory()
+        hostWq = t["Wq"].cpu().pin_memory()
+        hostWk = t["Wk"].cpu().pin_memory()
+        hostO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        dQ, dK, dV = torch.empty_like(t["Q"]), torch.empty_like(t["K"]), torch.empty_like(t["V"])
+        dWq, dWk = torch.empty_like(t["Wq"]), torch.empty_like(t["Wk"])
+        fws = vb.alloc_workspace(prob, dev)
+
+        def e2e_step():
+            dQ.copy_(hostQ, non_blocking=True)
+            dK.copy_(hostK, non_blocking=True)
+            dV.copy_(hostV, non_blocking=True)
+            dWq.copy_(hostWq, non_blocking=True)
+            dWk.copy_(hostWk, non_blocking=True)
+            vb.veda_forward(prob, dQ, dK, dV, dWq, dWk, O, None, None, None, fws)
+            hostO.copy_(O, non_blocking=True)
+
+        for _ in range(min(2, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(2, min(args.steps, 5))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        _barrier(world)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        _barrier(world)
+        e_ms = _max_over_ranks(a.elapsed_time(b) / n_e2e, world)
+        h2d = sum(x.numel() * x.element_size() for x in (hostQ, hostK, hostV, hostWq, hostWk))
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": hostO.numel() * hostO.element_size()}
+        del hostQ, hostK, hostV, hostO, dQ, dK, dV
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        th = {n: workloads.bf16_bits(t[n].index_select(1, torch.tensor([0], device=dev)))
+              for n in ("Q", "K", "V")}
+        th["Wq"], th["Wk"] = t["Wq"].cpu().numpy(), t["Wk"].cpu().numpy()
+        res = oracle_sample(w, th, heads=1, units_per_head=24)
+        cpu = {"value": flops / res["full_layer_s"] / 1e12, "unit": "TFLOP/s",
+               "cores": res["cores"], "kind": "oracle", "sample": res["sample"],
+               "seconds_sampled": res["seconds_sampled"],
+               "full_layer_s_extrapolated": res["full_layer_s"]}
+
+    if rank == 0:
+        peak = peaks["bf16_sus"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(w.describe(), parallelism="replicas (one layer per GPU)" if world > 1
+                           else "single GPU", l2="inputs larger than L2 (Q/K/V 6.0 GB)"),
+            "ms_per_layer": ms,
+            "frac_of_peak": {"measured_bf16_burst": value / world / peaks["bf16"],
+                             "measured_bf16_sustained": value / world / peaks["bf16_sus"],
+                             "datasheet_dense_bf16_2250": value / world / 2250.0,
+                             "peaks": peaks["source"]},
+            "roofline": {"bound": "tensor", "kernel": "sparse_attn", "achieved": attn_tf,
+                         "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
+                         "peak_kind": "bf16 sustained (" + peaks["source"] + ")",
+                         "frac_of_burst": attn_tf / peaks["bf16"], "traffic": None,
+                         "algorithmic_flops_per_launch": flops},
+            "kernels_ms": per,
+            "mask_prep": mask_prep,
+            "dense_path": {"attn_ms": dense_ms,
+                           "speedup_attention": (dense_ms / per["sparse_attn"]) if dense_ms else None,
+                           "speedup_layer": (dense_ms / ms) if dense_ms else None},
+            "device_status": status,
+            "gpu_launches": (nk + 1) * args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["veda", "reference"], default="veda")
+    ap.add_argument("--workload", default="long_video",
+                    help="long_video | 720p | 480p | tiny | sweep:T:sparsity")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "veda":
+        args.warmup = 3
+    if args.workload.startswith("sweep:"):
+        _, T, s = args.workload.split(":")
+        w = workloads.sweep(int(T), int(s))
+    else:
+        w = workloads.CONFIGS[args.workload]()
+    world, rank, local = _dist_init()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, w, world, rank)
+        return run_veda(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

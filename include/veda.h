@@ -1,0 +1,166 @@
+/*
+ * veda.h -- C ABI of the B200 (sm_100a) tile-sparse attention library.
+ *
+ * The library implements the inference hot path of Veda, "Veda: Scalable Video
+ * Diffusion via Distilled Sparse Attention" (project page), per head:
+ *   1. TripPool tile statistics (avg, max, min of Q and K over each tile);
+ *   2. tile scores through head-specific Q/K projections;
+ *   3. per query-tile Top-k into a tile mask / index list;
+ *   4. tile-skipping attention that reads only the selected K/V tiles.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer except `veda_problem::tile_shapes` is a caller-owned DEVICE
+ *   pointer.  The library never allocates, frees or keeps a pointer after the
+ *   call returns.  All work is enqueued asynchronously on `stream`; results are
+ *   ready when the stream reaches that point.
+ * - Tensors are dense and row-major.  Q, K, V, O are bf16 (passed as uint16_t
+ *   bit patterns) of shape [B, H, N, d] with N = T*Hs*Ws tokens in raster
+ *   (t, y, x) order: token n = (t*Hs + y)*Ws + x.
+ * - Head h uses the tile shape tile_shapes[h] = (p_t, p_h, p_w): tile j is the
+ *   p_t x p_h x p_w box of the token grid at tile-grid position
+ *   (a, b, c) with j = (a*(Hs/p_h) + b)*(Ws/p_w) + c.  Every head has the same
+ *   tile size Bt = p_t*p_h*p_w, so every head has nT = N/Bt tiles.
+ * - Supported: d in {64, 128}; Bt in {64, 128}; 1 <= k <= nT; H <= 256; at most
+ *   4 distinct tile shapes per call; nT <= 16384.  Other sizes return
+ *   VEDA_ERR_UNSUPPORTED before anything is launched.
+ * - Device pointers must be 16-byte aligned (VEDA_ERR_ALIGN otherwise).
+ * - A call that returns anything but VEDA_OK has launched nothing.
+ *   `veda_last_error()` then describes the failure (thread-local string).
+ * - Calls that take `ws` use its first VEDA_STATUS_BYTES bytes as a device
+ *   status word: they clear it, and a kernel that detects an error (a bounded
+ *   wait that gave up, an index-list entry out of range) writes its code there.
+ *   `veda_get_status` reads it back.
+ */
+#ifndef VEDA_H
+#define VEDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA stream type (identical to cudaStream_t / CUstream). */
+typedef struct CUstream_st* veda_stream_t;
+
+typedef enum veda_status {
+    VEDA_OK = 0,
+    VEDA_ERR_INVALID_ARG = 1,  /* null pointer, k out of range, bad scale */
+    VEDA_ERR_SHAPE = 2,        /* grid not divisible by a tile shape, tile sizes differ */
+    VEDA_ERR_UNSUPPORTED = 3,  /* d, Bt, H, nT or number of distinct shapes out of range */
+    VEDA_ERR_ALIGN = 4,        /* a device pointer is not 16-byte aligned */
+    VEDA_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed */
+    VEDA_ERR_TIMEOUT = 6,      /* device: a bounded wait gave up (read via veda_get_status) */
+    VEDA_ERR_BAD_INDEX = 7     /* device: an index-list entry was outside [0, nT) */
+} veda_status;
+
+/* Bytes at the start of every workspace that hold the device status word. */
+#define VEDA_STATUS_BYTES 256
+
+typedef struct veda_problem {
+    int64_t B;                  /* batch */
+    int64_t H;                  /* heads */
+    int64_t d;                  /* head dimension: 64 or 128 */
+    int64_t T, Hs, Ws;          /* latent grid (frames, height, width) */
+    const int32_t* tile_shapes; /* HOST pointer, [H][3] = (p_t, p_h, p_w) per head */
+    int64_t k;                  /* key tiles kept per query-tile row */
+    float scale;                /* softmax scale on q.k; 0 means 1/sqrt(d) */
+} veda_problem;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int veda_version(void);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* veda_last_error(void);
+
+/*
+ * Workspace bytes needed by veda_forward (a superset of what veda_tile_score
+ * and veda_sparse_attn need): status word, TripPool statistics, projected
+ * statistics, the score matrix and an index list.
+ */
+veda_status veda_workspace_size(const veda_problem* p, size_t* bytes);
+
+/*
+ * TripPool (project page, "Attention Structure Distillation", Estimator;
+ * "Theoretical Rationale" 2, Tile Statistics): per head, tile and channel, the
+ * average, maximum and minimum of Q (and of K) over the tile's Bt tokens.
+ *   Q, K          : bf16 [B, H, N, d]
+ *   statsQ, statsK: fp32 [B, H, nT, 3, d], statistic order (avg, max, min);
+ *                   avg is the fp32 sum divided by Bt; max and min are exact.
+ */
+veda_status veda_tripool(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
+                         float* statsQ, float* statsK, veda_stream_t stream);
+
+/*
+ * Tile score (project page, "Attention Structure Distillation", Estimator:
+ * head-specific Q/K projections of the statistics; "Theoretical Rationale" 4:
+ * the estimator's scores over key tiles before Top-k):
+ *   q~_{i,s} = statsQ[i,s,:] . Wq[h],  k~_{j,s} = statsK[j,s,:] . Wk[h],
+ *   S[i, j]  = sum over s in {avg, max, min} of <q~_{i,s}, k~_{j,s}>.
+ *   Wq, Wk: fp32 [H, d, d] (row = input channel, column = output channel)
+ *   S     : fp32 [B, H, nT, nT]
+ *   ws    : device workspace of at least
+ *           VEDA_STATUS_BYTES + 2 * B*H*nT*3*d*4 bytes (projected statistics).
+ * Arithmetic is fp32.
+ */
+veda_status veda_tile_score(const veda_problem* p, const float* statsQ, const float* statsK,
+                            const float* Wq, const float* Wk, float* S, void* ws,
+                            veda_stream_t stream);
+
+/*
+ * Head-aware Top-k (project page, "Attention Structure Distillation",
+ * Execution): for every query-tile row of S keep the k largest scores; ties go
+ * to the lower tile index, -0.0 ties with +0.0 (scores must be finite).
+ *   S   : fp32 [B, H, nT, nT]
+ *   mask: uint8 [B, H, nT, nT] of 0/1, may be NULL
+ *   idx : int32 [B, H, nT, k], the kept tile indices in ascending order
+ */
+veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask, int32_t* idx,
+                           veda_stream_t stream);
+
+/*
+ * Tile-skipping attention (project page, "Attention Structure Distillation",
+ * Execution and "Principle 03 Tile-Sparse Kernel"; "Theoretical Rationale" 1:
+ * the kept keys are renormalised among themselves).  For every query token of
+ * tile i of head h:
+ *   O   = softmax(scale * q.k over every key of the tiles idx[b,h,i,:]) . V
+ *   lse = ln sum exp(scale * q.k) over the same keys
+ *   idx: int32 [B, H, nT, k] tile indices in [0, nT) (each row's entries should
+ *        be distinct; order does not matter), or NULL for the dense schedule
+ *        (every tile, k taken as nT).
+ *   O  : bf16 [B, H, N, d];  lse: fp32 [B, H, N] or NULL
+ *   ws : device workspace of at least VEDA_STATUS_BYTES bytes
+ * bf16 tensor-core products with fp32 accumulation and an fp32 softmax; P is
+ * rounded to bf16 before the P.V product.  An out-of-range index is replaced
+ * by tile 0 and reported as VEDA_ERR_BAD_INDEX in the status word.
+ */
+veda_status veda_sparse_attn(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
+                             const uint16_t* V, const int32_t* idx, uint16_t* O, float* lse,
+                             void* ws, veda_stream_t stream);
+
+/*
+ * The whole layer: TripPool -> projection and score -> Top-k -> tile-skipping
+ * attention, all on `stream`.
+ *   idx_out : int32 [B, H, nT, k] or NULL (then held in ws)
+ *   mask_out: uint8 [B, H, nT, nT] or NULL
+ *   lse     : fp32 [B, H, N] or NULL
+ *   ws      : at least veda_workspace_size() bytes
+ */
+veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
+                         const uint16_t* V, const float* Wq, const float* Wk, uint16_t* O,
+                         float* lse, int32_t* idx_out, uint8_t* mask_out, void* ws,
+                         veda_stream_t stream);
+
+/*
+ * Waits for `stream`, then copies the device status word of `ws` into
+ * *device_status (VEDA_OK or a device-detected veda_status code).
+ */
+veda_status veda_get_status(const void* ws, veda_stream_t stream, int32_t* device_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VEDA_H */

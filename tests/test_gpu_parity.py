@@ -1,0 +1,251 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the fp64 oracle.
+
+Every test draws seeded synthetic inputs once and feeds the same tensors to
+both sides.  Small workloads are compared element by element; the large ones
+(720P-like, 245K-token long video, sweep points) on sampled heads / query
+tiles that the oracle computes one by one, in the launch configuration the
+benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import parity_helpers as ph
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def vb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import tile_sparse_attention_b200 as m
+    m.load_library()
+    return m
+
+
+def _inputs(w, device):
+    t = workloads.generate(w, device=device)
+    return {n: (v.cuda() if v.device.type != "cuda" else v) for n, v in t.items()}
+
+
+def _bits(t):
+    return ph.to_host_bits(t)
+
+
+# ------------------------------------------------------------------ mask prep
+@pytest.mark.parametrize("make,heads", [(workloads.tiny, None), (workloads.p480, None),
+                                        (workloads.p720, [0, 7, 21, 39])])
+def test_tripool_and_score_parity(vb, oracle, make, heads):
+    w = make()
+    t = _inputs(w, "cuda")
+    prob = vb.Problem.from_workload(w)
+    g = ph.gpu_mask_prep(vb, prob, t["Q"], t["K"], t["Wq"], t["Wk"])
+    heads = list(range(w.H)) if heads is None else heads
+    Qb, Kb = _bits(t["Q"]), _bits(t["K"])
+    Wq, Wk = t["Wq"].cpu().numpy(), t["Wk"].cpu().numpy()
+    ora = ph.oracle_mask_prep_heads(oracle, w, Qb, Kb, Wq, Wk, heads)
+    ph.check_stats(g["statsQ"][:, heads].cpu().numpy(), ora["statsQ"], w.Bt)
+    ph.check_stats(g["statsK"][:, heads].cpu().numpy(), ora["statsK"], w.Bt)
+    S_gpu = g["S"][:, heads].cpu().numpy().astype(np.float64)
+    bound = ph.score_bound(ora, Wq[heads], Wk[heads])
+    err = np.abs(S_gpu - ora["S"])
+    assert np.all(err <= bound), f"score error {err.max()} (bound {bound.min()})"
+    ph.check_masks(g["mask"][:, heads].cpu().numpy(), g["idx"][:, heads].cpu().numpy(),
+                   ora["S"], ora["mask"], ora["idx"], w.k)
+
+
+def test_topk_bit_exact_on_given_scores(vb, oracle):
+    """Same fp32 scores on both sides (ties, -0.0/+0.0, ragged nT): identical selection."""
+    rng = np.random.default_rng(7)
+    for nT, k in ((240, 24), (37, 5), (600, 30), (8, 8), (1920, 96), (33, 1), (5000, 250)):
+        w = workloads.custom("topk", 1, 3, 64, (1, 1, 64 * nT), [(1, 1, 64)], k)
+        S = rng.standard_normal((1, 3, nT, nT)).astype(np.float32)
+        S[:, :, :, ::5] = S[:, :, :, :1]          # exact ties across columns
+        S[:, 0, :, 1] = -0.0
+        S[:, 0, :, 2] = 0.0
+        S[:, 1] = np.round(S[:, 1] * 4) / 4       # many ties
+        prob = vb.Problem.from_workload(w)
+        St = torch.from_numpy(S).cuda()
+        mask = torch.empty((1, 3, nT, nT), dtype=torch.uint8, device="cuda")
+        idx = torch.empty((1, 3, nT, k), dtype=torch.int32, device="cuda")
+        vb.veda_topk_mask(prob, St, mask, idx)
+        m_o, i_o = oracle.topk(S.astype(np.float64), k)
+        np.testing.assert_array_equal(idx.cpu().numpy(), i_o)
+        np.testing.assert_array_equal(mask.cpu().numpy(), m_o)
+
+
+# ------------------------------------------------------------------ attention
+def _attn_case(vb, oracle, w, t, idx_np, units, dense=False):
+    prob = vb.Problem.from_workload(w)
+    if units is None:
+        units = np.array([(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(w.nT)],
+                         dtype=np.int64)
+    if idx_np is None:
+        idx_np = np.broadcast_to(np.arange(w.nT, dtype=np.int32), (w.B, w.H, w.nT, w.nT)).copy()
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    ws = vb.alloc_workspace(prob)
+    idx_t = None if dense else torch.from_numpy(idx_np).cuda()
+    vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx_t, O, lse, ws)
+    assert vb.veda_get_status(ws) == 0
+    Qb, Kb, Vb = _bits(t["Q"]), _bits(t["K"]), _bits(t["V"])
+    O_o, lse_o, toks = oracle.sparse_attention(Qb, Kb, Vb, idx_np, w.grid, w.tile_shapes,
+                                               w.scale, units=units)
+    return ph.check_attention(_bits(O), lse.cpu().numpy(), units, O_o, lse_o, toks), O, lse
+
+
+@pytest.mark.parametrize("make,per_head", [(workloads.tiny, None), (workloads.p480, 6)])
+def test_sparse_attn_parity(vb, oracle, make, per_head):
+    w = make()
+    t = _inputs(w, "cuda")
+    Qb, Kb = _bits(t["Q"]), _bits(t["K"])
+    ora = oracle.mask_prep(Qb, Kb, t["Wq"].cpu().numpy(), t["Wk"].cpu().numpy(), w.grid,
+                           w.tile_shapes, w.k)
+    units = None if per_head is None else workloads.sample_units(w, per_head, seed=1)
+    _attn_case(vb, oracle, w, t, ora["idx"], units)
+
+
+def test_sparse_attn_head_aware_shapes_and_batch(vb, oracle):
+    """Three tile shapes across heads, B = 2, random index lists (unsorted rows)."""
+    grid = (8, 16, 32)
+    shapes = [(1, 8, 16), (2, 8, 8), (4, 4, 8), (2, 8, 8)]
+    w = workloads.custom("mixed", 2, 4, 128, grid, shapes, 7)
+    t = _inputs(w, "cuda")
+    rng = np.random.default_rng(3)
+    idx = np.stack([rng.permutation(w.nT)[:w.k] for _ in range(w.B * w.H * w.nT)])
+    idx = idx.reshape(w.B, w.H, w.nT, w.k).astype(np.int32)
+    units = workloads.sample_units(w, 5, seed=2)
+    _attn_case(vb, oracle, w, t, idx, units)
+
+
+@pytest.mark.parametrize("d,shape", [(64, (1, 8, 8)), (128, (1, 8, 8)), (64, (2, 8, 8)),
+                                     (128, (4, 4, 8))])
+def test_sparse_attn_dims_and_tile_sizes(vb, oracle, d, shape):
+    grid = (4, 16, 32)
+    w = workloads.custom("dims", 1, 2, d, grid, [shape], 3)
+    t = _inputs(w, "cuda")
+    rng = np.random.default_rng(d)
+    idx = np.sort(np.stack([rng.permutation(w.nT)[:w.k] for _ in range(w.H * w.nT)]), 1)
+    idx = idx.reshape(1, w.H, w.nT, w.k).astype(np.int32)
+    _attn_case(vb, oracle, w, t, idx, None)
+
+
+def test_k_equals_all_tiles_is_dense_path(vb, oracle):
+    """k = nT through an index list equals the dense schedule bit for bit, and the oracle."""
+    w = workloads.custom("dense", 1, 2, 128, (4, 16, 32), [(2, 8, 8)], 16)
+    t = _inputs(w, "cuda")
+    idx = np.broadcast_to(np.arange(w.nT, dtype=np.int32), (1, w.H, w.nT, w.nT)).copy()
+    _, O1, l1 = _attn_case(vb, oracle, w, t, idx, None)
+    _, O2, l2 = _attn_case(vb, oracle, w, t, None, None, dense=True)
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+
+
+def test_k_one(vb, oracle):
+    w = workloads.custom("k1", 1, 2, 128, (4, 16, 32), [(1, 8, 16)], 1)
+    t = _inputs(w, "cuda")
+    idx = np.random.default_rng(0).integers(0, w.nT, (1, w.H, w.nT, 1)).astype(np.int32)
+    _attn_case(vb, oracle, w, t, idx, None)
+
+
+def test_bad_index_reported(vb):
+    w = workloads.custom("bad", 1, 1, 128, (2, 8, 16), [(1, 8, 16)], 2)
+    t = _inputs(w, "cuda")
+    prob = vb.Problem.from_workload(w)
+    idx = torch.zeros((1, 1, w.nT, 2), dtype=torch.int32, device="cuda")
+    idx[0, 0, 0, 1] = w.nT + 5
+    O = torch.empty_like(t["Q"])
+    ws = vb.alloc_workspace(prob)
+    vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O, None, ws)
+    assert vb.veda_get_status(ws) == 7  # VEDA_ERR_BAD_INDEX
+
+
+# ------------------------------------------------------------------ whole layer
+def _forward(vb, w, t, want_mask=True):
+    prob = vb.Problem.from_workload(w)
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    idx = torch.empty((w.B, w.H, w.nT, w.k), dtype=torch.int32, device="cuda")
+    mask = torch.empty((w.B, w.H, w.nT, w.nT), dtype=torch.uint8, device="cuda") \
+        if want_mask else None
+    ws = vb.alloc_workspace(prob)
+    vb.veda_forward(prob, t["Q"], t["K"], t["V"], t["Wq"], t["Wk"], O, lse, idx, mask, ws)
+    assert vb.veda_get_status(ws) == 0
+    return O, lse, idx, mask
+
+
+def _forward_parity(vb, oracle, w, heads, per_head, device="cuda"):
+    t = _inputs(w, device)
+    O, lse, idx, mask = _forward(vb, w, t)
+    # heads are independent: the oracle runs on the selected heads only
+    sel = torch.tensor(heads, device="cuda")
+    Qb, Kb, Vb = (_bits(t[n].index_select(1, sel)) for n in ("Q", "K", "V"))
+    Wq, Wk = t["Wq"].cpu().numpy()[heads], t["Wk"].cpu().numpy()[heads]
+    shapes = [w.tile_shapes[h] for h in heads]
+    ora = oracle.mask_prep(Qb, Kb, Wq, Wk, w.grid, shapes, w.k)
+    idx_g = idx.index_select(1, sel).cpu().numpy()
+    ph.check_masks(mask.index_select(1, sel).cpu().numpy(), idx_g, ora["S"], ora["mask"],
+                   ora["idx"], w.k)
+    # attention on sampled query tiles; the oracle gets the (verified) GPU index list
+    units = workloads.sample_units(w, per_head, seed=4)
+    hmap = {h: n for n, h in enumerate(heads)}
+    units = np.array([(b, hmap[int(h)], i) for b, h, i in units if int(h) in hmap],
+                     dtype=np.int64)
+    O_o, lse_o, toks = oracle.sparse_attention(Qb, Kb, Vb, idx_g, w.grid, shapes, w.scale,
+                                               units=units)
+    return ph.check_attention(_bits(O.index_select(1, sel)),
+                              lse.index_select(1, sel).cpu().numpy(), units, O_o, lse_o, toks)
+
+
+def test_forward_tiny(vb, oracle):
+    w = workloads.tiny()
+    _forward_parity(vb, oracle, w, list(range(w.H)), w.nT, device="cpu")
+
+
+def test_forward_480p(vb, oracle):
+    w = workloads.p480()
+    _forward_parity(vb, oracle, w, list(range(w.H)), 6, device="cpu")
+
+
+def test_forward_720p(vb, oracle):
+    w = workloads.p720()
+    _forward_parity(vb, oracle, w, [0, 13, 26, 39], 6)
+
+
+def test_forward_long_video(vb, oracle):
+    """245,760 tokens, 1,920 tiles, k = 96: full-size launch, sampled heads and tiles."""
+    w = workloads.long_video()
+    _forward_parity(vb, oracle, w, [0, 31], 4)
+
+
+@pytest.mark.parametrize("T,s", [(4, 0), (4, 98), (8, 50), (20, 80), (32, 90), (64, 95)])
+def test_forward_sweep_points(vb, oracle, T, s):
+    w = workloads.sweep(T, s)
+    _forward_parity(vb, oracle, w, [0, 23], 3)
+
+
+def test_sweep_k_all_matches_dense_path(vb):
+    """Sweep 0% sparsity: veda_forward with k = nT equals the dense schedule exactly."""
+    w = workloads.sweep(4, 0)
+    t = _inputs(w, "cuda")
+    O, lse, idx, _ = _forward(vb, w, t, want_mask=False)
+    prob = vb.Problem.from_workload(w)
+    O2 = torch.empty_like(O)
+    lse2 = torch.empty_like(lse)
+    ws = vb.alloc_workspace(prob)
+    vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], None, O2, lse2, ws)
+    assert vb.veda_get_status(ws) == 0
+    assert torch.equal(O, O2) and torch.equal(lse, lse2)
+    assert torch.equal(idx[0, 0, 0].cpu(), torch.arange(w.nT, dtype=torch.int32))
+
+
+def test_forward_is_deterministic(vb):
+    w = workloads.p480()
+    t = _inputs(w, "cuda")
+    a = _forward(vb, w, t)
+    b = _forward(vb, w, t)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)

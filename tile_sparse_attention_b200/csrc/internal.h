@@ -1,0 +1,57 @@
+// internal.h -- shared host-side declarations of the library (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/veda.h"
+
+namespace veda {
+
+constexpr int kMaxHeads = 256;
+constexpr int kMaxShapes = 4;
+constexpr int64_t kMaxTiles = 16384;
+
+// Validated view of a veda_problem.
+struct Problem {
+    int B, H, d, T, Hs, Ws, N, Bt, nT, k;
+    float scale;
+    int nshapes;                  // distinct tile shapes
+    int shape[kMaxShapes][3];     // (p_t, p_h, p_w) per distinct shape
+    int head_shape[kMaxHeads];    // head -> distinct-shape slot
+};
+
+// Records a message for veda_last_error() and returns `code`.
+veda_status fail(veda_status code, const std::string& msg);
+
+// Validates `p` (k is checked only when need_k).
+veda_status make_problem(const veda_problem* p, bool need_k, Problem* out);
+
+veda_status check_ptr(const void* ptr, const char* name, bool nullable = false);
+
+veda_status cuda_check(cudaError_t err, const char* what);
+
+// Launchers (defined next to their kernels).  Each returns VEDA_OK or an
+// error after checking the launch.
+veda_status launch_tripool(const Problem& pr, const uint16_t* Q, const uint16_t* K, float* statsQ,
+                           float* statsK, cudaStream_t s);
+veda_status launch_project(const Problem& pr, const float* stats, const float* W, float* out,
+                           cudaStream_t s);
+veda_status launch_score(const Problem& pr, const float* qt, const float* kt, float* S,
+                         cudaStream_t s);
+veda_status launch_topk(const Problem& pr, const float* S, uint8_t* mask, int32_t* idx,
+                        cudaStream_t s);
+veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint16_t* K,
+                               const uint16_t* V, const int32_t* idx, int k, uint16_t* O,
+                               float* lse, int* status, cudaStream_t s);
+
+// Workspace layout of veda_forward (byte offsets, 256-aligned).
+struct WorkspaceLayout {
+    size_t status, statsQ, statsK, qt, kt, S, idx, total;
+};
+WorkspaceLayout workspace_layout(const Problem& pr);
+
+}  // namespace veda

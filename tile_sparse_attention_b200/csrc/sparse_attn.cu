@@ -1,0 +1,580 @@
+// sparse_attn.cu -- tile-skipping flash attention for sm_100a (tcgen05 + TMEM + TMA).
+//
+// "Veda: Scalable Video Diffusion via Distilled Sparse Attention" (project
+// page): "Attention Structure Distillation", Execution (the tile mask is
+// passed to a tile-skipping kernel that fetches only the selected K/V tiles);
+// "Principle 03 Tile-Sparse Kernel" (selected K/V tiles arrive by TMA and the
+// gathers overlap the tensor-core products); "Theoretical Rationale" 1
+// (Softmax Geometry: the kept keys are renormalised among themselves).
+//
+// The page's kernel targets Hopper (warpgroup MMA); this one is written for
+// Blackwell:
+//   * one CTA per query tile (b, h, i); 256 threads in four roles:
+//       warp 0      TMA producer: the Q tile once, then for every selected key
+//                   tile j the K and V tiles into an NS-deep ring.  A tile is a
+//                   p_t x p_h x p_w box of the token grid, fetched by a 5-D TMA
+//                   copy (d, Ws, Hs, T, B*H) with a 64-channel, 128-byte-swizzled
+//                   box, so no gather kernel or token permutation is needed;
+//       warp 1      allocates tensor memory; lane 0 issues every tcgen05.mma:
+//                   S_j = Q K_j^T into one of two TMEM S buffers, and
+//                   O += P_j V_j into the TMEM O accumulator;
+//       warps 4..7  softmax: thread r owns query row r, reads S_j from TMEM,
+//                   keeps the running max / sum in fp32 (exp2 with the scale
+//                   folded in), writes P_j as bf16 into shared memory in the
+//                   MMA operand layout, and rescales O in TMEM only when the
+//                   running max grows by more than 2^8 (exact: the final
+//                   normalisation uses the same max);
+//   * S_{j+1} is computed while the softmax works on S_j, and P_j V_j runs
+//     while the softmax computes the exponentials of tile j+1;
+//   * the epilogue normalises O, stages it in shared memory and writes it back
+//     with the same 5-D box through a TMA store; lse is written per token.
+// Every wait on an mbarrier is bounded by a time limit; on expiry the CTA sets
+// VEDA_ERR_TIMEOUT in the status word, drains its outstanding copies and
+// tensor-core work (again with a limit), frees its tensor memory and exits.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace veda {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct __align__(64) AttnParams {
+    CUtensorMap tmQ[kMaxShapes];
+    CUtensorMap tmK[kMaxShapes];
+    CUtensorMap tmV[kMaxShapes];
+    CUtensorMap tmO[kMaxShapes];
+    int shape[kMaxShapes][3];
+    unsigned char head_shape[kMaxHeads];
+    const int32_t* idx;  // [B,H,nT,k] or null (dense schedule)
+    float* lse;          // [B,H,N] or null
+    int* status;
+    int H, T, Hs, Ws, N, nT, k;
+    float scale_log2;
+    unsigned long long wait_limit_ns;
+};
+
+template <int D, int BT, int NS>
+struct Cfg {
+    static constexpr int kChunks = D / 64;           // 64-channel (128-byte) chunks
+    static constexpr int kQBytes = 128 * D * 2;      // Q padded to the 128-row MMA tile
+    static constexpr int kQChunk = 128 * 128;        // bytes per Q chunk (128 rows x 128 B)
+    static constexpr int kKVBytes = BT * D * 2;      // one K or V tile
+    static constexpr int kKVChunk = BT * 128;        // bytes per K/V chunk
+    static constexpr int kPBytes = 128 * BT * 2;     // P: 128 rows x BT keys
+    static constexpr int kPChunk = 128 * 128;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kQBytes;
+    static constexpr int kOffV = kOffK + NS * kKVBytes;
+    static constexpr int kOffP = kOffV + NS * kKVBytes;
+    static constexpr int kOffBar = kOffP + kPBytes;
+    // barriers: q, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS], s_full[2],
+    // s_free[2], p_full, o_done, drain
+    static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 3;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    static constexpr int kTmemS = 0;                 // S buffers at columns [0, 2 BT)
+    static constexpr int kTmemO = 2 * BT;            // O at columns [2 BT, 2 BT + D)
+    static constexpr int kTmemCols = (2 * BT + D) <= 256 ? 256 : 512;
+    static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, BT, false);
+    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+};
+
+struct Bars {
+    uint64_t* q;
+    uint64_t* k_full;
+    uint64_t* v_full;
+    uint64_t* k_empty;
+    uint64_t* v_empty;
+    uint64_t* s_full;
+    uint64_t* s_free;
+    uint64_t* p_full;
+    uint64_t* o_done;
+    uint64_t* drain;
+};
+
+// Bounded wait: false when the limit expired or another role aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const AttnParams& p,
+                                         volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > p.wait_limit_ns) {
+            *abort_flag = 1;
+            atomicCAS(p.status, 0, (int)VEDA_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag (drain on the way out).
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity, const AttnParams& p) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > p.wait_limit_ns) {
+            atomicCAS(p.status, 0, (int)VEDA_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast and the
+// warp re-converges (the thread sync orders the other lanes after the wait).
+__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
+                                              const AttnParams& p, volatile int* abort_flag) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, p, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+__device__ __forceinline__ void tile_origin(int t, int pt, int ph, int pw, int Hs, int Ws,
+                                            int& t0, int& y0, int& x0) {
+    const int nh = Hs / ph, nw = Ws / pw;
+    t0 = (t / (nh * nw)) * pt;
+    y0 = ((t / nw) % nh) * ph;
+    x0 = (t % nw) * pw;
+}
+
+template <int D, int BT, int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_kernel(const __grid_constant__ AttnParams p) {
+    using C = Cfg<D, BT, NS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sQ = smem + C::kOffQ;
+    uint8_t* sK = smem + C::kOffK;
+    uint8_t* sV = smem + C::kOffV;
+    uint8_t* sP = smem + C::kOffP;
+    uint64_t* bar_base = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    Bars bars;
+    bars.q = bar_base;
+    bars.k_full = bar_base + 1;
+    bars.v_full = bars.k_full + NS;
+    bars.k_empty = bars.v_full + NS;
+    bars.v_empty = bars.k_empty + NS;
+    bars.s_full = bars.v_empty + NS;
+    bars.s_free = bars.s_full + 2;
+    bars.p_full = bars.s_free + 2;
+    bars.o_done = bars.p_full + 1;
+    bars.drain = bars.o_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i_tile = blockIdx.x;
+    const int bh = blockIdx.y;
+    const int h = bh % p.H;
+    const int slot = p.head_shape[h];
+    const int pt = p.shape[slot][0], ph = p.shape[slot][1], pw = p.shape[slot][2];
+    const int k = p.k;
+
+    // ---------------------------------------------------------------- set-up
+    if (threadIdx.x == 0) {
+        mbar_init(bars.q, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&bars.k_full[s], 1);
+            mbar_init(&bars.v_full[s], 1);
+            mbar_init(&bars.k_empty[s], 1);
+            mbar_init(&bars.v_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.s_full[b], 1);
+            mbar_init(&bars.s_free[b], 4);
+        }
+        mbar_init(bars.p_full, 4);
+        mbar_init(bars.o_done, 1);
+        mbar_init(bars.drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (BT < 128) {
+        // rows BT..127 of the padded Q operand are zero
+        for (int c = 0; c < C::kChunks; ++c) {
+            uint4* q = reinterpret_cast<uint4*>(sQ + c * C::kQChunk + BT * 128);
+            for (int e = threadIdx.x; e < (128 - BT) * 8; e += kThreads) q[e] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == 0) {
+        // ============================================================ producer
+        int i_t0, i_y0, i_x0;
+        tile_origin(i_tile, pt, ph, pw, p.Hs, p.Ws, i_t0, i_y0, i_x0);
+        const int32_t* irow = p.idx ? p.idx + ((size_t)bh * p.nT + i_tile) * k : nullptr;
+        int k_fills = 0, v_fills = 0;  // K / V tiles issued (lane 0)
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tmQ[slot]);
+            tma_prefetch_desc(&p.tmK[slot]);
+            tma_prefetch_desc(&p.tmV[slot]);
+            mbar_arrive_expect_tx(bars.q, BT * D * 2);
+#pragma unroll
+            for (int c = 0; c < C::kChunks; ++c)
+                tma_load_5d(sQ + c * C::kQChunk, &p.tmQ[slot], bars.q, c * 64, i_x0, i_y0, i_t0, bh);
+        }
+        bool ok = true;
+        for (int j0 = 0; j0 < k && ok; j0 += 32) {
+            int my_t = 0;
+            if (j0 + lane < k) {
+                my_t = irow ? irow[j0 + lane] : j0 + lane;
+                if (my_t < 0 || my_t >= p.nT) {
+                    atomicCAS(p.status, 0, (int)VEDA_ERR_BAD_INDEX);
+                    my_t = 0;
+                }
+            }
+            const int cnt = min(32, k - j0);
+            for (int jj = 0; jj < cnt; ++jj) {
+                const int t = __shfl_sync(0xffffffffu, my_t, jj);
+                int good = 1;
+                if (lane == 0) {
+                    const int j = j0 + jj, st = j % NS, n = j / NS;
+                    int t0, y0, x0;
+                    tile_origin(t, pt, ph, pw, p.Hs, p.Ws, t0, y0, x0);
+                    if (n > 0) good = wait_bar(&bars.k_empty[st], (n - 1) & 1, p, abort_flag);
+                    if (good) {
+                        mbar_arrive_expect_tx(&bars.k_full[st], C::kKVBytes);
+#pragma unroll
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_5d(sK + st * C::kKVBytes + c * C::kKVChunk, &p.tmK[slot],
+                                        &bars.k_full[st], c * 64, x0, y0, t0, bh);
+                        k_fills = j + 1;
+                        if (n > 0) good = wait_bar(&bars.v_empty[st], (n - 1) & 1, p, abort_flag);
+                        if (good) {
+                            mbar_arrive_expect_tx(&bars.v_full[st], C::kKVBytes);
+#pragma unroll
+                            for (int c = 0; c < C::kChunks; ++c)
+                                tma_load_5d(sV + st * C::kKVBytes + c * C::kKVChunk, &p.tmV[slot],
+                                            &bars.v_full[st], c * 64, x0, y0, t0, bh);
+                            v_fills = j + 1;
+                        }
+                    }
+                }
+                good = __shfl_sync(0xffffffffu, good, 0);
+                if (!good) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        if (lane == 0) {
+            // Drain: every copy this warp issued has landed before the CTA exits.
+            drain_bar(bars.q, 0, p);
+            for (int st = 0; st < NS; ++st) {
+                // the last fill of stage st is tile st + m*NS < fills
+                if (st < k_fills)
+                    drain_bar(&bars.k_full[st], (((k_fills - 1 - st) / NS)) & 1, p);
+                if (st < v_fills)
+                    drain_bar(&bars.v_full[st], (((v_fills - 1 - st) / NS)) & 1, p);
+            }
+        }
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        if (lane == 0) {
+            const uint32_t tS = tbase + C::kTmemS;
+            const uint32_t tO = tbase + C::kTmemO;
+            const uint32_t q_addr = smem_addr(sQ);
+            const uint32_t k_addr = smem_addr(sK);
+            const uint32_t v_addr = smem_addr(sV);
+            const uint32_t p_addr = smem_addr(sP);
+            bool ok = wait_bar(bars.q, 0, p, abort_flag);
+            auto issue_qk = [&](int j) -> bool {
+                const int st = j % NS;
+                if (!wait_bar(&bars.k_full[st], (j / NS) & 1, p, abort_flag)) return false;
+                if (j >= 2 && !wait_bar(&bars.s_free[j & 1], ((j - 2) >> 1) & 1, p, abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t d_tmem = tS + (j & 1) * BT;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const int c = ks >> 2, w = ks & 3;
+                    const uint64_t a = smem_desc_sw128(q_addr + c * C::kQChunk + w * 32, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(
+                        k_addr + st * C::kKVBytes + c * C::kKVChunk + w * 32, 16, 1024);
+                    mma_bf16_ss(d_tmem, a, b, C::kIdescQK, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars.s_full[j & 1]);
+                mma_commit(&bars.k_empty[st]);
+                return true;
+            };
+            if (ok) ok = issue_qk(0);
+            for (int j = 0; j < k && ok; ++j) {
+                if (j + 1 < k && !issue_qk(j + 1)) {
+                    ok = false;
+                    break;
+                }
+                const int st = j % NS;
+                if (!wait_bar(bars.p_full, j & 1, p, abort_flag)) break;
+                if (!wait_bar(&bars.v_full[st], (j / NS) & 1, p, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < BT / 16; ++ks) {
+                    const int c = ks >> 2, w = ks & 3;
+                    const uint64_t a = smem_desc_sw128(p_addr + c * C::kPChunk + w * 32, 16, 1024);
+                    const uint64_t b =
+                        smem_desc_sw128(v_addr + st * C::kKVBytes + ks * 2048, C::kKVChunk, 1024);
+                    mma_bf16_ss(tO, a, b, C::kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+                }
+                mma_commit(bars.o_done);
+                mma_commit(&bars.v_empty[st]);
+            }
+            // Drain: all tensor-core work issued by this thread has completed.
+            mma_commit(bars.drain);
+            drain_bar(bars.drain, 0, p);
+        }
+        __syncwarp();
+    } else if (warp >= kSoftmaxWarp0) {
+        // ============================================================ softmax
+        const int wq = warp & 3;                 // TMEM lane quarter of this warp
+        const int r = wq * 32 + lane;            // query row of the tile
+        const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tbase + lane_off + C::kTmemS;
+        const uint32_t tO = tbase + lane_off + C::kTmemO;
+        const float c2 = p.scale_log2;
+        float m_run = 0.f, l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < k; ++j) {
+            if (!warp_wait_bar(&bars.s_full[j & 1], (j >> 1) & 1, p, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t s[BT];
+#pragma unroll
+            for (int cc = 0; cc < BT / 32; ++cc)
+                tmem_ld_32x32b_x32(tS + (j & 1) * BT + cc * 32,
+                                   *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
+
+            float mx = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < BT; ++e) mx = fmaxf(mx, __uint_as_float(s[e]));
+            const float m_tile = mx * c2;
+            bool need;
+            float m_use, alpha;
+            if (j == 0) {
+                need = false;
+                m_use = m_tile;
+                alpha = 0.f;
+            } else {
+                const float m_new = fmaxf(m_run, m_tile);
+                need = m_new > m_run + kRescaleThreshold;
+                m_use = need ? m_new : m_run;
+                alpha = need ? fast_exp2(m_run - m_new) : 1.f;
+            }
+            uint32_t pk[BT / 2];
+            float lsum = 0.f;
+#pragma unroll
+            for (int e = 0; e < BT; e += 2) {
+                const float p0 = fast_exp2(fmaf(__uint_as_float(s[e]), c2, -m_use));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(s[e + 1]), c2, -m_use));
+                lsum += p0 + p1;
+                pk[e / 2] = pack_bf16x2(p0, p1);
+            }
+            l_run = (j == 0) ? lsum : fmaf(l_run, alpha, lsum);
+            m_run = m_use;
+
+            if (j > 0) {
+                // P_{j-1} V_{j-1} has finished: the P buffer is free and O is stable.
+                if (!warp_wait_bar(bars.o_done, (j - 1) & 1, p, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(tO + cc * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st_32x32b_x32(tO + cc * 32, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row r -> shared memory, K-major 128-byte-swizzled operand layout.
+#pragma unroll
+            for (int u = 0; u < BT / 8; ++u) {
+                const int c = u >> 3, uc = u & 7;
+                uint4 v = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                *reinterpret_cast<uint4*>(sP + c * C::kPChunk + r * 128 + ((uc ^ (r & 7)) << 4)) = v;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.p_full);
+        }
+        if (ok) ok = warp_wait_bar(bars.o_done, (k - 1) & 1, p, abort_flag);
+        // every softmax thread gets here (all waits are bounded); the epilogue
+        // runs only if all four warps finished their loop
+        if (named_barrier_and(1, 128, ok)) {
+            tc_fence_after();
+            // ---------------------------------------------------- epilogue
+            const float inv_l = 1.f / l_run;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(tO + cc * 32, o);
+                tmem_wait_ld();
+                const int c = cc >> 1;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int uc = (cc & 1) * 4 + q;
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l,
+                                      __uint_as_float(o[8 * q + 1]) * inv_l);
+                    v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l,
+                                      __uint_as_float(o[8 * q + 3]) * inv_l);
+                    v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l,
+                                      __uint_as_float(o[8 * q + 5]) * inv_l);
+                    v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l,
+                                      __uint_as_float(o[8 * q + 7]) * inv_l);
+                    *reinterpret_cast<uint4*>(sQ + c * C::kQChunk + r * 128 + ((uc ^ (r & 7)) << 4)) = v;
+                }
+            }
+            fence_proxy_async_smem();
+            named_barrier_sync(2, 128);
+            int i_t0, i_y0, i_x0;
+            tile_origin(i_tile, pt, ph, pw, p.Hs, p.Ws, i_t0, i_y0, i_x0);
+            if (threadIdx.x == kSoftmaxWarp0 * 32) {
+#pragma unroll
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_store_5d(&p.tmO[slot], sQ + c * C::kQChunk, c * 64, i_x0, i_y0, i_t0, bh);
+                bulk_commit_group();
+                bulk_wait_group_all();
+            }
+            if (p.lse != nullptr && r < BT) {
+                const int lt = r / (ph * pw), lh = (r / pw) % ph, lw = r % pw;
+                const int n = ((i_t0 + lt) * p.Hs + (i_y0 + lh)) * p.Ws + (i_x0 + lw);
+                p.lse[(size_t)bh * p.N + n] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 5-D view (d, Ws, Hs, T, B*H) of a [B,H,N,d] bf16 tensor; box (64, pw, ph, pt, 1).
+veda_status encode_tile_map(CUtensorMap* map, const void* base, const Problem& pr,
+                            const int* shape) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (enc == nullptr) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[5] = {(cuuint64_t)pr.d, (cuuint64_t)pr.Ws, (cuuint64_t)pr.Hs,
+                                (cuuint64_t)pr.T, (cuuint64_t)pr.B * pr.H};
+    const cuuint64_t strides[4] = {(cuuint64_t)pr.d * 2, (cuuint64_t)pr.Ws * pr.d * 2,
+                                   (cuuint64_t)pr.Hs * pr.Ws * pr.d * 2,
+                                   (cuuint64_t)pr.N * pr.d * 2};
+    const cuuint32_t box[5] = {64, (cuuint32_t)shape[2], (cuuint32_t)shape[1],
+                               (cuuint32_t)shape[0], 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string((int)r));
+    return VEDA_OK;
+}
+
+template <int D, int BT, int NS>
+veda_status launch_cfg(const AttnParams& prm, const Problem& pr, cudaStream_t s) {
+    using C = Cfg<D, BT, NS>;
+    static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
+    cudaError_t err = cudaFuncSetAttribute(sparse_attn_kernel<D, BT, NS>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           C::kSmemBytes);
+    if (err != cudaSuccess) return cuda_check(err, "sparse_attn smem attribute");
+    dim3 grid(pr.nT, pr.B * pr.H);
+    sparse_attn_kernel<D, BT, NS><<<grid, kThreads, C::kSmemBytes, s>>>(prm);
+    return cuda_check(cudaGetLastError(), "sparse_attn launch");
+}
+
+unsigned long long wait_limit_ns() {
+    const char* env = getenv("VEDA_WAIT_LIMIT_MS");
+    unsigned long long ms = 10000ull;  // a healthy wait takes microseconds
+    if (env != nullptr && atoll(env) > 0) ms = (unsigned long long)atoll(env);
+    return ms * 1000000ull;
+}
+
+}  // namespace
+
+veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint16_t* K,
+                               const uint16_t* V, const int32_t* idx, int k, uint16_t* O,
+                               float* lse, int* status, cudaStream_t s) {
+    AttnParams prm;
+    memset(&prm, 0, sizeof(prm));
+    for (int sh = 0; sh < pr.nshapes; ++sh) {
+        veda_status st;
+        if ((st = encode_tile_map(&prm.tmQ[sh], Q, pr, pr.shape[sh])) != VEDA_OK) return st;
+        if ((st = encode_tile_map(&prm.tmK[sh], K, pr, pr.shape[sh])) != VEDA_OK) return st;
+        if ((st = encode_tile_map(&prm.tmV[sh], V, pr, pr.shape[sh])) != VEDA_OK) return st;
+        if ((st = encode_tile_map(&prm.tmO[sh], O, pr, pr.shape[sh])) != VEDA_OK) return st;
+        for (int q = 0; q < 3; ++q) prm.shape[sh][q] = pr.shape[sh][q];
+    }
+    for (int h = 0; h < pr.H; ++h) prm.head_shape[h] = (unsigned char)pr.head_shape[h];
+    prm.idx = idx;
+    prm.lse = lse;
+    prm.status = status;
+    prm.H = pr.H;
+    prm.T = pr.T;
+    prm.Hs = pr.Hs;
+    prm.Ws = pr.Ws;
+    prm.N = pr.N;
+    prm.nT = pr.nT;
+    prm.k = k;
+    prm.scale_log2 = pr.scale * 1.4426950408889634f;
+    prm.wait_limit_ns = wait_limit_ns();
+    if (pr.d == 128 && pr.Bt == 128) return launch_cfg<128, 128, 2>(prm, pr, s);
+    if (pr.d == 128 && pr.Bt == 64) return launch_cfg<128, 64, 3>(prm, pr, s);
+    if (pr.d == 64 && pr.Bt == 128) return launch_cfg<64, 128, 3>(prm, pr, s);
+    return launch_cfg<64, 64, 4>(prm, pr, s);
+}
+
+}  // namespace veda

@@ -1,0 +1,188 @@
+// tile_score.cu -- head-specific projection of the TripPool statistics and the
+// tile-pair score matrix.
+//
+// "Veda: Scalable Video Diffusion via Distilled Sparse Attention" (project
+// page), "Attention Structure Distillation", Estimator: head-specific Q/K
+// projections reconstruct the dense tile distribution from the average,
+// maximum and minimum statistics; "Theoretical Rationale" 4: the estimator
+// yields a score for every key tile before Top-k.
+//
+//   projection: q~[b,h] (3nT x d) = statsQ[b,h] (3nT x d) . Wq[h] (d x d)
+//   score     : S[b,h] (nT x nT)  = q~[b,h] (nT x 3d) . k~[b,h]^T
+//
+// Both are small fp32 contractions (fp32 keeps the Top-k decision stable, so
+// they run on the FP32 SIMT pipes): one batched register-blocked SGEMM kernel,
+// 128 x 128 block tile, 8 x 8 outputs per thread, double-buffered shared
+// memory.  ALU-bound at ~75 TFLOP/s of FP32 FMA peak.
+#include "internal.h"
+
+namespace veda {
+
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 8, PAD = 4;
+
+struct GemmParams {
+    const float* A;
+    const float* B;
+    float* C;
+    int M, N, K;
+    int lda, ldb, ldc;
+    long long strideA, strideB, strideC;  // per batch entry
+    int b_batch_mod;                      // >0: B index = batch % b_batch_mod
+};
+
+// C[z] = A[z] . B[z]  (B_T = false: B is K x N row-major)
+// C[z] = A[z] . B[z]^T (B_T = true: B is N x K row-major)
+template <bool B_T>
+__global__ void __launch_bounds__(256) sgemm_kernel(const __grid_constant__ GemmParams p) {
+    __shared__ __align__(16) float As[2][BK][BM + PAD];
+    __shared__ __align__(16) float Bs[2][BK][BN + PAD];
+
+    const int z = blockIdx.z;
+    const float* A = p.A + (long long)z * p.strideA;
+    const int bz = p.b_batch_mod > 0 ? z % p.b_batch_mod : z;
+    const float* Bm = p.B + (long long)bz * p.strideB;
+    float* C = p.C + (long long)z * p.strideC;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+
+    // global -> register staging
+    const int a_row = tid >> 1, a_k = (tid & 1) * 4;
+    const int bn_k = tid >> 5, bn_n = (tid & 31) * 4;  // B not transposed
+    float4 ra, rb;
+
+    auto load_a = [&](int k0) {
+        const int m = m0 + a_row;
+        ra = (m < p.M) ? *reinterpret_cast<const float4*>(A + (long long)m * p.lda + k0 + a_k)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    auto load_b = [&](int k0) {
+        if (B_T) {
+            const int n = n0 + a_row;
+            rb = (n < p.N) ? *reinterpret_cast<const float4*>(Bm + (long long)n * p.ldb + k0 + a_k)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            const int n = n0 + bn_n;
+            rb = (n < p.N)
+                     ? *reinterpret_cast<const float4*>(Bm + (long long)(k0 + bn_k) * p.ldb + n)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto store_tiles = [&](int buf) {
+        As[buf][a_k + 0][a_row] = ra.x;
+        As[buf][a_k + 1][a_row] = ra.y;
+        As[buf][a_k + 2][a_row] = ra.z;
+        As[buf][a_k + 3][a_row] = ra.w;
+        if (B_T) {
+            Bs[buf][a_k + 0][a_row] = rb.x;
+            Bs[buf][a_k + 1][a_row] = rb.y;
+            Bs[buf][a_k + 2][a_row] = rb.z;
+            Bs[buf][a_k + 3][a_row] = rb.w;
+        } else {
+            *reinterpret_cast<float4*>(&Bs[buf][bn_k][bn_n]) = rb;
+        }
+    };
+
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+    load_a(0);
+    load_b(0);
+    store_tiles(0);
+    __syncthreads();
+    const int nk = p.K / BK;
+    for (int kt = 0; kt < nk; ++kt) {
+        const int buf = kt & 1;
+        if (kt + 1 < nk) {
+            load_a((kt + 1) * BK);
+            load_b((kt + 1) * BK);
+        }
+#pragma unroll
+        for (int kk = 0; kk < BK; ++kk) {
+            const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        if (kt + 1 < nk) {
+            store_tiles(buf ^ 1);
+            __syncthreads();
+        }
+    }
+
+    const bool vec = (p.ldc % 4) == 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+        if (m >= p.M) continue;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int n = n0 + half * 64 + tx * 4;
+            float* dst = C + (long long)m * p.ldc + n;
+            const float* v = &acc[i][half * 4];
+            if (vec && n + 3 < p.N) {
+                *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+            } else {
+                for (int e = 0; e < 4; ++e)
+                    if (n + e < p.N) dst[e] = v[e];
+            }
+        }
+    }
+}
+
+}  // namespace
+
+veda_status launch_project(const Problem& pr, const float* stats, const float* W, float* out,
+                           cudaStream_t s) {
+    GemmParams g{};
+    g.A = stats;
+    g.B = W;
+    g.C = out;
+    g.M = 3 * pr.nT;
+    g.N = pr.d;
+    g.K = pr.d;
+    g.lda = pr.d;
+    g.ldb = pr.d;
+    g.ldc = pr.d;
+    g.strideA = (long long)3 * pr.nT * pr.d;
+    g.strideB = (long long)pr.d * pr.d;
+    g.strideC = g.strideA;
+    g.b_batch_mod = pr.H;
+    dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM, pr.B * pr.H);
+    sgemm_kernel<false><<<grid, 256, 0, s>>>(g);
+    return cuda_check(cudaGetLastError(), "projection launch");
+}
+
+veda_status launch_score(const Problem& pr, const float* qt, const float* kt, float* S,
+                         cudaStream_t s) {
+    GemmParams g{};
+    g.A = qt;
+    g.B = kt;
+    g.C = S;
+    g.M = pr.nT;
+    g.N = pr.nT;
+    g.K = 3 * pr.d;
+    g.lda = 3 * pr.d;
+    g.ldb = 3 * pr.d;
+    g.ldc = pr.nT;
+    g.strideA = (long long)3 * pr.nT * pr.d;
+    g.strideB = g.strideA;
+    g.strideC = (long long)pr.nT * pr.nT;
+    g.b_batch_mod = 0;
+    dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM, pr.B * pr.H);
+    sgemm_kernel<true><<<grid, 256, 0, s>>>(g);
+    return cuda_check(cudaGetLastError(), "score launch");
+}
+
+}  // namespace veda

@@ -1,0 +1,246 @@
+// veda_api.cu -- the C ABI (include/veda.h): argument validation, workspace
+// layout and the composition of the four kernels into the layer call.
+//
+// "Veda: Scalable Video Diffusion via Distilled Sparse Attention" (project
+// page), "Attention Structure Distillation": TripPool and the head-specific
+// projections (Estimator) feed a head-aware Top-k whose tile mask drives the
+// tile-skipping kernel (Execution).
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "internal.h"
+
+namespace veda {
+
+namespace {
+thread_local std::string g_last_error;
+}
+
+veda_status fail(veda_status code, const std::string& msg) {
+    g_last_error = msg;
+    return code;
+}
+
+veda_status cuda_check(cudaError_t err, const char* what) {
+    if (err == cudaSuccess) return VEDA_OK;
+    return fail(VEDA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(err));
+}
+
+veda_status check_ptr(const void* ptr, const char* name, bool nullable) {
+    if (ptr == nullptr) {
+        if (nullable) return VEDA_OK;
+        return fail(VEDA_ERR_INVALID_ARG, std::string(name) + " is NULL");
+    }
+    if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0)
+        return fail(VEDA_ERR_ALIGN, std::string(name) + " is not 16-byte aligned");
+    return VEDA_OK;
+}
+
+veda_status make_problem(const veda_problem* p, bool need_k, Problem* out) {
+    if (p == nullptr) return fail(VEDA_ERR_INVALID_ARG, "problem is NULL");
+    if (p->tile_shapes == nullptr) return fail(VEDA_ERR_INVALID_ARG, "tile_shapes is NULL");
+    if (p->B < 1 || p->H < 1 || p->T < 1 || p->Hs < 1 || p->Ws < 1)
+        return fail(VEDA_ERR_INVALID_ARG, "B, H, T, Hs and Ws must be >= 1");
+    if (p->d != 64 && p->d != 128) return fail(VEDA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if (p->H > kMaxHeads) return fail(VEDA_ERR_UNSUPPORTED, "at most 256 heads");
+    const int64_t N = p->T * p->Hs * p->Ws;
+    if (N > (1ll << 30) || p->B * p->H > 65535)
+        return fail(VEDA_ERR_UNSUPPORTED, "token count or B*H too large");
+    Problem& pr = *out;
+    memset(&pr, 0, sizeof(pr));
+    pr.B = (int)p->B;
+    pr.H = (int)p->H;
+    pr.d = (int)p->d;
+    pr.T = (int)p->T;
+    pr.Hs = (int)p->Hs;
+    pr.Ws = (int)p->Ws;
+    pr.N = (int)N;
+    pr.nshapes = 0;
+    int Bt = -1;
+    for (int h = 0; h < pr.H; ++h) {
+        const int32_t* s = p->tile_shapes + 3 * h;
+        if (s[0] < 1 || s[1] < 1 || s[2] < 1)
+            return fail(VEDA_ERR_SHAPE, "tile shape entries must be >= 1");
+        if (p->T % s[0] || p->Hs % s[1] || p->Ws % s[2])
+            return fail(VEDA_ERR_SHAPE, "grid not divisible by the tile shape of head " +
+                                            std::to_string(h));
+        const int bt = s[0] * s[1] * s[2];
+        if (Bt < 0) Bt = bt;
+        if (bt != Bt) return fail(VEDA_ERR_SHAPE, "tile sizes p_t*p_h*p_w differ between heads");
+        int slot = -1;
+        for (int q = 0; q < pr.nshapes; ++q)
+            if (pr.shape[q][0] == s[0] && pr.shape[q][1] == s[1] && pr.shape[q][2] == s[2]) slot = q;
+        if (slot < 0) {
+            if (pr.nshapes == kMaxShapes)
+                return fail(VEDA_ERR_UNSUPPORTED, "more than 4 distinct tile shapes");
+            slot = pr.nshapes++;
+            pr.shape[slot][0] = s[0];
+            pr.shape[slot][1] = s[1];
+            pr.shape[slot][2] = s[2];
+        }
+        pr.head_shape[h] = slot;
+    }
+    if (Bt != 64 && Bt != 128) return fail(VEDA_ERR_UNSUPPORTED, "tile size must be 64 or 128");
+    pr.Bt = Bt;
+    pr.nT = pr.N / Bt;
+    if (pr.nT > kMaxTiles) return fail(VEDA_ERR_UNSUPPORTED, "more than 16384 tiles per head");
+    if (need_k && (p->k < 1 || p->k > pr.nT))
+        return fail(VEDA_ERR_INVALID_ARG, "k must be in [1, nT]");
+    pr.k = (int)p->k;
+    float scale = p->scale;
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)pr.d);
+    if (!(scale > 0.f) || !isfinite(scale))
+        return fail(VEDA_ERR_INVALID_ARG, "scale must be positive and finite (0 = 1/sqrt(d))");
+    pr.scale = scale;
+    return VEDA_OK;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+WorkspaceLayout workspace_layout(const Problem& pr) {
+    WorkspaceLayout w{};
+    const size_t stats = (size_t)pr.B * pr.H * pr.nT * 3 * pr.d * sizeof(float);
+    size_t off = 0;
+    w.status = off;
+    off += VEDA_STATUS_BYTES;
+    w.qt = off;  // tile_score's own workspace follows the status word
+    off = align256(off + stats);
+    w.kt = off;
+    off = align256(off + stats);
+    w.statsQ = off;
+    off = align256(off + stats);
+    w.statsK = off;
+    off = align256(off + stats);
+    w.S = off;
+    off = align256(off + (size_t)pr.B * pr.H * pr.nT * pr.nT * sizeof(float));
+    w.idx = off;
+    off = align256(off + (size_t)pr.B * pr.H * pr.nT * pr.k * sizeof(int32_t));
+    w.total = off;
+    return w;
+}
+
+}  // namespace veda
+
+using namespace veda;
+
+extern "C" {
+
+int veda_version(void) { return 10000; }
+
+const char* veda_last_error(void) { return g_last_error.c_str(); }
+
+veda_status veda_workspace_size(const veda_problem* p, size_t* bytes) {
+    Problem pr;
+    veda_status st = make_problem(p, true, &pr);
+    if (st != VEDA_OK) return st;
+    if (bytes == nullptr) return fail(VEDA_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = workspace_layout(pr).total;
+    return VEDA_OK;
+}
+
+veda_status veda_tripool(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
+                         float* statsQ, float* statsK, veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, false, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(Q, "Q")) || (st = check_ptr(K, "K")) || (st = check_ptr(statsQ, "statsQ")) ||
+        (st = check_ptr(statsK, "statsK")))
+        return st;
+    return launch_tripool(pr, Q, K, statsQ, statsK, (cudaStream_t)stream);
+}
+
+veda_status veda_tile_score(const veda_problem* p, const float* statsQ, const float* statsK,
+                            const float* Wq, const float* Wk, float* S, void* ws,
+                            veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, false, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(statsQ, "statsQ")) || (st = check_ptr(statsK, "statsK")) ||
+        (st = check_ptr(Wq, "Wq")) || (st = check_ptr(Wk, "Wk")) || (st = check_ptr(S, "S")) ||
+        (st = check_ptr(ws, "ws")))
+        return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const WorkspaceLayout w = workspace_layout(pr);
+    char* base = static_cast<char*>(ws);
+    float* qt = reinterpret_cast<float*>(base + w.qt);
+    float* kt = reinterpret_cast<float*>(base + w.kt);
+    if ((st = cuda_check(cudaMemsetAsync(base + w.status, 0, sizeof(int), s), "status reset")))
+        return st;
+    if ((st = launch_project(pr, statsQ, Wq, qt, s))) return st;
+    if ((st = launch_project(pr, statsK, Wk, kt, s))) return st;
+    return launch_score(pr, qt, kt, S, s);
+}
+
+veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask, int32_t* idx,
+                           veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, true, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(S, "S")) || (st = check_ptr(idx, "idx")) ||
+        (st = check_ptr(mask, "mask", true)))
+        return st;
+    return launch_topk(pr, S, mask, idx, (cudaStream_t)stream);
+}
+
+veda_status veda_sparse_attn(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
+                             const uint16_t* V, const int32_t* idx, uint16_t* O, float* lse,
+                             void* ws, veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, idx != nullptr, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(Q, "Q")) || (st = check_ptr(K, "K")) || (st = check_ptr(V, "V")) ||
+        (st = check_ptr(O, "O")) || (st = check_ptr(idx, "idx", true)) ||
+        (st = check_ptr(lse, "lse", true)) || (st = check_ptr(ws, "ws")))
+        return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    int* status = static_cast<int*>(ws);
+    if ((st = cuda_check(cudaMemsetAsync(status, 0, sizeof(int), s), "status reset"))) return st;
+    const int k = idx ? pr.k : pr.nT;
+    return launch_sparse_attn(pr, Q, K, V, idx, k, O, lse, status, s);
+}
+
+veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
+                         const uint16_t* V, const float* Wq, const float* Wk, uint16_t* O,
+                         float* lse, int32_t* idx_out, uint8_t* mask_out, void* ws,
+                         veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, true, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(Q, "Q")) || (st = check_ptr(K, "K")) || (st = check_ptr(V, "V")) ||
+        (st = check_ptr(Wq, "Wq")) || (st = check_ptr(Wk, "Wk")) || (st = check_ptr(O, "O")) ||
+        (st = check_ptr(lse, "lse", true)) || (st = check_ptr(idx_out, "idx_out", true)) ||
+        (st = check_ptr(mask_out, "mask_out", true)) || (st = check_ptr(ws, "ws")))
+        return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const WorkspaceLayout w = workspace_layout(pr);
+    char* base = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(base + w.status);
+    float* statsQ = reinterpret_cast<float*>(base + w.statsQ);
+    float* statsK = reinterpret_cast<float*>(base + w.statsK);
+    float* qt = reinterpret_cast<float*>(base + w.qt);
+    float* kt = reinterpret_cast<float*>(base + w.kt);
+    float* S = reinterpret_cast<float*>(base + w.S);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+    if ((st = cuda_check(cudaMemsetAsync(status, 0, sizeof(int), s), "status reset"))) return st;
+    if ((st = launch_tripool(pr, Q, K, statsQ, statsK, s))) return st;
+    if ((st = launch_project(pr, statsQ, Wq, qt, s))) return st;
+    if ((st = launch_project(pr, statsK, Wk, kt, s))) return st;
+    if ((st = launch_score(pr, qt, kt, S, s))) return st;
+    if ((st = launch_topk(pr, S, mask_out, idx, s))) return st;
+    return launch_sparse_attn(pr, Q, K, V, idx, pr.k, O, lse, status, s);
+}
+
+veda_status veda_get_status(const void* ws, veda_stream_t stream, int32_t* device_status) {
+    if (ws == nullptr || device_status == nullptr)
+        return fail(VEDA_ERR_INVALID_ARG, "ws and device_status must be non-NULL");
+    veda_status st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((st = cuda_check(cudaStreamSynchronize(s), "stream synchronize"))) return st;
+    return cuda_check(cudaMemcpy(device_status, ws, sizeof(int32_t), cudaMemcpyDeviceToHost),
+                      "status read");
+}
+
+}  // extern "C"
