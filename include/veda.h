@@ -159,6 +159,32 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
  */
 veda_status veda_get_status(const void* ws, veda_stream_t stream, int32_t* device_status);
 
+/*
+ * The paper has no counterpart for the two calls below; they exist for
+ * callers that cannot allocate device memory (an application that only
+ * receives device pointers for its inputs and outputs from another runtime, a
+ * plugin whose host forbids allocations after start-up, a real-time loop that
+ * must not call cudaMalloc because it can synchronise the device).
+ *
+ * veda_tile_score_noalloc computes exactly what veda_tile_score computes, but
+ * keeps its scratch (status word and projected statistics) in a fixed device
+ * array inside the library instead of a caller workspace:
+ *   - the array holds veda_noalloc_scratch_bytes() bytes (64 MiB); every GPU
+ *     that loads the library keeps it until the process exits;
+ *   - a problem needing more than VEDA_STATUS_BYTES + 2*B*H*nT*3*d*4 bytes of
+ *     it returns VEDA_ERR_UNSUPPORTED and launches nothing;
+ *   - the first call on a device looks up the array's address on that device
+ *     (the device must be current); make that first call before any stream
+ *     capture;
+ *   - all calls share the array: calls whose work overlaps on the GPU race;
+ *     each call clears the status word it uses;
+ *   - it allocates nothing (no cudaMalloc, no cudaFree).
+ */
+size_t veda_noalloc_scratch_bytes(void);
+veda_status veda_tile_score_noalloc(const veda_problem* p, const float* statsQ,
+                                    const float* statsK, const float* Wq, const float* Wk,
+                                    float* S, veda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

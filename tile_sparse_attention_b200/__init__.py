@@ -71,6 +71,9 @@ def load_library(path: str = LIB_PATH):
     lib.veda_forward.restype = st
     lib.veda_get_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32)]
     lib.veda_get_status.restype = st
+    lib.veda_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.veda_tile_score_noalloc.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 6
+    lib.veda_tile_score_noalloc.restype = st
     _lib = lib
     return lib
 
@@ -185,6 +188,21 @@ def veda_get_status(ws, stream=None) -> int:
     out = ctypes.c_int32(0)
     _check(load_library().veda_get_status(_ptr(ws), _stream(stream), ctypes.byref(out)))
     return int(out.value)
+
+
+def veda_tile_score_noalloc(problem: Problem, statsQ, statsK, Wq, Wk, S, stream=None) -> None:
+    """veda_tile_score without a workspace, for callers that cannot allocate device
+    memory: the library's fixed scratch array (veda_noalloc_scratch_bytes()) is
+    used instead.  Calls that overlap on the GPU race on that array."""
+    for t, n in ((statsQ, "statsQ"), (statsK, "statsK"), (Wq, "Wq"), (Wk, "Wk"), (S, "S")):
+        _expect(t, torch.float32, n)
+    _check(load_library().veda_tile_score_noalloc(ctypes.byref(problem.c), _ptr(statsQ),
+                                                  _ptr(statsK), _ptr(Wq), _ptr(Wk), _ptr(S),
+                                                  _stream(stream)))
+
+
+def veda_noalloc_scratch_bytes() -> int:
+    return int(load_library().veda_noalloc_scratch_bytes())
 
 
 def alloc_workspace(problem: Problem, device="cuda") -> torch.Tensor:
