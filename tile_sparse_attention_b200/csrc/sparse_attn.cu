@@ -11,21 +11,25 @@
 // Blackwell:
 //   * one CTA per query tile (b, h, i); 256 threads in four roles:
 //       warp 0      TMA producer: the Q tile once, then for every selected key
-//                   tile j the K and V tiles into an NS-deep ring.  A tile is a
+//                   tile j the K and V tiles into NS-deep rings.  A tile is a
 //                   p_t x p_h x p_w box of the token grid, fetched by a 5-D TMA
 //                   copy (d, Ws, Hs, T, B*H) with a 64-channel, 128-byte-swizzled
 //                   box, so no gather kernel or token permutation is needed;
 //       warp 1      allocates tensor memory; lane 0 issues every tcgen05.mma:
-//                   S_j = Q K_j^T into one of two TMEM S buffers, and
-//                   O += P_j V_j into the TMEM O accumulator;
-//       warps 4..7  softmax: thread r owns query row r, reads S_j from TMEM,
+//                   S_j = Q K_j^T and O += P_j V_j, both with the A operand (Q,
+//                   P_j) read from tensor memory and B (K_j, V_j) from shared
+//                   memory, so shared memory only carries the K and V tiles (an
+//                   M=128, N=128 product with both operands in shared memory
+//                   would use its whole bandwidth);
+//       warps 4..7  softmax: thread r owns query row r; copies its Q row into
+//                   tensor memory once; then per tile reads S_j from TMEM,
 //                   keeps the running max / sum in fp32 (exp2 with the scale
-//                   folded in), writes P_j as bf16 into shared memory in the
-//                   MMA operand layout, and rescales O in TMEM only when the
-//                   running max grows by more than 2^8 (exact: the final
-//                   normalisation uses the same max);
+//                   folded in, packed fp32x2 arithmetic), writes P_j as bf16
+//                   into one of two TMEM P buffers, and rescales O in TMEM only
+//                   when the running max grows by more than 2^8 (exact: the
+//                   final normalisation uses the same max);
 //   * S_{j+1} is computed while the softmax works on S_j, and P_j V_j runs
-//     while the softmax computes the exponentials of tile j+1;
+//     while the softmax works on S_{j+1};
 //   * the epilogue normalises O, stages it in shared memory and writes it back
 //     with the same 5-D box through a TMA store; lse is written per token.
 // Every wait on an mbarrier is bounded by a time limit; on expiry the CTA sets
@@ -62,31 +66,33 @@ struct __align__(64) AttnParams {
 template <int D, int BT, int NS>
 struct Cfg {
     static constexpr int kChunks = D / 64;           // 64-channel (128-byte) chunks
-    static constexpr int kQBytes = 128 * D * 2;      // Q padded to the 128-row MMA tile
-    static constexpr int kQChunk = 128 * 128;        // bytes per Q chunk (128 rows x 128 B)
+    static constexpr int kQChunk = 128 * 128;        // bytes per Q staging chunk (128 rows x 128 B)
+    static constexpr int kQBytes = kChunks * kQChunk;
     static constexpr int kKVBytes = BT * D * 2;      // one K or V tile
     static constexpr int kKVChunk = BT * 128;        // bytes per K/V chunk
-    static constexpr int kPBytes = 128 * BT * 2;     // P: 128 rows x BT keys
-    static constexpr int kPChunk = 128 * 128;
-    static constexpr int kOffQ = 0;
+    static constexpr int kOffQ = 0;                  // Q staging, later O staging
     static constexpr int kOffK = kQBytes;
     static constexpr int kOffV = kOffK + NS * kKVBytes;
-    static constexpr int kOffP = kOffV + NS * kKVBytes;
-    static constexpr int kOffBar = kOffP + kPBytes;
-    // barriers: q, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS], s_full[2],
-    // s_free[2], p_full, o_done, drain
-    static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 3;
+    static constexpr int kOffBar = kOffV + NS * kKVBytes;
+    // barriers: q, q_tmem, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS],
+    // s_full, s_free, p_full[2], p_free[2], drain
+    static constexpr int kNumBars = 2 + 4 * NS + 1 + 1 + 2 + 2 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-    static constexpr int kTmemS = 0;                 // S buffers at columns [0, 2 BT)
-    static constexpr int kTmemO = 2 * BT;            // O at columns [2 BT, 2 BT + D)
-    static constexpr int kTmemCols = (2 * BT + D) <= 256 ? 256 : 512;
+    // tensor memory columns (all offsets multiples of 64)
+    static constexpr int kTmemS = 0;                 // S_j, fp32, BT columns
+    static constexpr int kTmemP = BT;                // P buffers: 2 x 64 columns of bf16 pairs
+    static constexpr int kTmemQ = BT + 128;          // Q: D/2 columns of bf16 pairs
+    static constexpr int kTmemO = BT + 192;          // O accumulator, fp32, D columns
+    static constexpr int kTmemCols = (kTmemO + D) <= 256 ? 256 : 512;
+    static_assert(kTmemO + D <= 512, "tensor memory budget");
     static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, BT, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
 };
 
 struct Bars {
     uint64_t* q;
+    uint64_t* q_tmem;
     uint64_t* k_full;
     uint64_t* v_full;
     uint64_t* k_empty;
@@ -94,7 +100,7 @@ struct Bars {
     uint64_t* s_full;
     uint64_t* s_free;
     uint64_t* p_full;
-    uint64_t* o_done;
+    uint64_t* p_free;
     uint64_t* drain;
 };
 
@@ -144,6 +150,18 @@ __device__ __forceinline__ void tile_origin(int t, int pt, int ph, int pw, int H
     x0 = (t % nw) * pw;
 }
 
+// Barrier phase bookkeeping (each barrier completes once per use):
+//   k_full/v_full[st]   fill n of stage st (tile j = st + n*NS): parity n & 1
+//   k_empty/v_empty[st] the MMA consumed fill n: parity n & 1
+//   s_full              QK_j done: parity j & 1
+//   s_free              softmax has read S_j: parity j & 1
+//   p_full[b]           P_j in TMEM (and O rescaled), j = b + 2m: parity m & 1
+//   p_free[b]           P_j V_j done, j = b + 2m: parity m & 1
+// For every barrier the next completion needs the waiter to have passed its
+// current wait, and no waiter skips a completion it has to see, so a waiter is
+// never two phases away from its barrier and the parities are unambiguous.
+// (P_j V_j completing is read from p_free: the softmax waits on P_{j-2} V_{j-2}
+// in every iteration, which keeps that barrier within one phase.)
 template <int D, int BT, int NS>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ AttnParams p) {
@@ -154,19 +172,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* sK = smem + C::kOffK;
     uint8_t* sV = smem + C::kOffV;
-    uint8_t* sP = smem + C::kOffP;
     uint64_t* bar_base = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     Bars bars;
     bars.q = bar_base;
-    bars.k_full = bar_base + 1;
+    bars.q_tmem = bar_base + 1;
+    bars.k_full = bar_base + 2;
     bars.v_full = bars.k_full + NS;
     bars.k_empty = bars.v_full + NS;
     bars.v_empty = bars.k_empty + NS;
     bars.s_full = bars.v_empty + NS;
-    bars.s_free = bars.s_full + 2;
-    bars.p_full = bars.s_free + 2;
-    bars.o_done = bars.p_full + 1;
-    bars.drain = bars.o_done + 1;
+    bars.s_free = bars.s_full + 1;
+    bars.p_full = bars.s_free + 1;
+    bars.p_free = bars.p_full + 2;
+    bars.drain = bars.p_free + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -181,29 +199,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- set-up
     if (threadIdx.x == 0) {
         mbar_init(bars.q, 1);
+        mbar_init(bars.q_tmem, 4);
         for (int s = 0; s < NS; ++s) {
             mbar_init(&bars.k_full[s], 1);
             mbar_init(&bars.v_full[s], 1);
             mbar_init(&bars.k_empty[s], 1);
             mbar_init(&bars.v_empty[s], 1);
         }
+        mbar_init(bars.s_full, 1);
+        mbar_init(bars.s_free, 4);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars.s_full[b], 1);
-            mbar_init(&bars.s_free[b], 4);
+            mbar_init(&bars.p_full[b], 4);
+            mbar_init(&bars.p_free[b], 1);
         }
-        mbar_init(bars.p_full, 4);
-        mbar_init(bars.o_done, 1);
         mbar_init(bars.drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (BT < 128) {
-        // rows BT..127 of the padded Q operand are zero
+        // rows BT..127 of the Q staging buffer are zero (they become zero rows of
+        // the 128-row MMA operand)
         for (int c = 0; c < C::kChunks; ++c) {
             uint4* q = reinterpret_cast<uint4*>(sQ + c * C::kQChunk + BT * 128);
             for (int e = threadIdx.x; e < (128 - BT) * 8; e += kThreads) q[e] = make_uint4(0, 0, 0, 0);
         }
-        fence_proxy_async_smem();
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -278,38 +297,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             drain_bar(bars.q, 0, p);
             for (int st = 0; st < NS; ++st) {
                 // the last fill of stage st is tile st + m*NS < fills
-                if (st < k_fills)
-                    drain_bar(&bars.k_full[st], (((k_fills - 1 - st) / NS)) & 1, p);
-                if (st < v_fills)
-                    drain_bar(&bars.v_full[st], (((v_fills - 1 - st) / NS)) & 1, p);
+                if (st < k_fills) drain_bar(&bars.k_full[st], ((k_fills - 1 - st) / NS) & 1, p);
+                if (st < v_fills) drain_bar(&bars.v_full[st], ((v_fills - 1 - st) / NS) & 1, p);
             }
         }
     } else if (warp == 1) {
         // ============================================================ MMA issuer
         if (lane == 0) {
             const uint32_t tS = tbase + C::kTmemS;
+            const uint32_t tP = tbase + C::kTmemP;
+            const uint32_t tQ = tbase + C::kTmemQ;
             const uint32_t tO = tbase + C::kTmemO;
-            const uint32_t q_addr = smem_addr(sQ);
             const uint32_t k_addr = smem_addr(sK);
             const uint32_t v_addr = smem_addr(sV);
-            const uint32_t p_addr = smem_addr(sP);
-            bool ok = wait_bar(bars.q, 0, p, abort_flag);
+            bool ok = wait_bar(bars.q_tmem, 0, p, abort_flag);
+            // S_j = Q K_j^T: A = Q from tensor memory, B = K tile (K-major, swizzled)
             auto issue_qk = [&](int j) -> bool {
                 const int st = j % NS;
                 if (!wait_bar(&bars.k_full[st], (j / NS) & 1, p, abort_flag)) return false;
-                if (j >= 2 && !wait_bar(&bars.s_free[j & 1], ((j - 2) >> 1) & 1, p, abort_flag))
-                    return false;
+                if (j >= 1 && !wait_bar(bars.s_free, (j - 1) & 1, p, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t d_tmem = tS + (j & 1) * BT;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const int c = ks >> 2, w = ks & 3;
-                    const uint64_t a = smem_desc_sw128(q_addr + c * C::kQChunk + w * 32, 16, 1024);
                     const uint64_t b = smem_desc_sw128(
                         k_addr + st * C::kKVBytes + c * C::kKVChunk + w * 32, 16, 1024);
-                    mma_bf16_ss(d_tmem, a, b, C::kIdescQK, ks > 0 ? 1u : 0u);
+                    mma_bf16_ts(tS, tQ + ks * 8, b, C::kIdescQK, ks > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars.s_full[j & 1]);
+                mma_commit(bars.s_full);
                 mma_commit(&bars.k_empty[st]);
                 return true;
             };
@@ -320,18 +335,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const int st = j % NS;
-                if (!wait_bar(bars.p_full, j & 1, p, abort_flag)) break;
+                if (!wait_bar(&bars.p_full[j & 1], (j >> 1) & 1, p, abort_flag)) break;
                 if (!wait_bar(&bars.v_full[st], (j / NS) & 1, p, abort_flag)) break;
                 tc_fence_after();
+                // O += P_j V_j: A = P_j from tensor memory, B = V tile (MN-major)
+                const uint32_t pa = tP + (j & 1) * 64;
 #pragma unroll
                 for (int ks = 0; ks < BT / 16; ++ks) {
-                    const int c = ks >> 2, w = ks & 3;
-                    const uint64_t a = smem_desc_sw128(p_addr + c * C::kPChunk + w * 32, 16, 1024);
                     const uint64_t b =
                         smem_desc_sw128(v_addr + st * C::kKVBytes + ks * 2048, C::kKVChunk, 1024);
-                    mma_bf16_ss(tO, a, b, C::kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+                    mma_bf16_ts(tO, pa + ks * 8, b, C::kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
                 }
-                mma_commit(bars.o_done);
+                mma_commit(&bars.p_free[j & 1]);
                 mma_commit(&bars.v_empty[st]);
             }
             // Drain: all tensor-core work issued by this thread has completed.
@@ -345,12 +360,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = wq * 32 + lane;            // query row of the tile
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tbase + lane_off + C::kTmemS;
+        const uint32_t tP = tbase + lane_off + C::kTmemP;
+        const uint32_t tQ = tbase + lane_off + C::kTmemQ;
         const uint32_t tO = tbase + lane_off + C::kTmemO;
         const float c2 = p.scale_log2;
         float m_run = 0.f, l_run = 0.f;
-        bool ok = true;
-        for (int j = 0; j < k; ++j) {
-            if (!warp_wait_bar(&bars.s_full[j & 1], (j >> 1) & 1, p, abort_flag)) {
+        bool ok = warp_wait_bar(bars.q, 0, p, abort_flag);
+        // lane 0 saw the Q copy land; each lane now observes the completed phase
+        // itself (one test, which succeeds) before reading the staged tile
+        if (ok) ok = __all_sync(0xffffffffu, mbar_try_wait(bars.q, 0));
+        if (ok) {
+            // Q row r: shared-memory staging (128-byte swizzle) -> tensor memory
+#pragma unroll
+            for (int c = 0; c < C::kChunks; ++c) {
+                uint32_t v[32];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(sQ + c * C::kQChunk + r * 128 +
+                                                                    ((u ^ (r & 7)) << 4));
+                    v[4 * u] = x.x;
+                    v[4 * u + 1] = x.y;
+                    v[4 * u + 2] = x.z;
+                    v[4 * u + 3] = x.w;
+                }
+                tmem_st_32x32b_x32(tQ + c * 32, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.q_tmem);
+        }
+        for (int j = 0; j < k && ok; ++j) {
+            if (!warp_wait_bar(bars.s_full, j & 1, p, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -358,16 +399,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t s[BT];
 #pragma unroll
             for (int cc = 0; cc < BT / 32; ++cc)
-                tmem_ld_32x32b_x32(tS + (j & 1) * BT + cc * 32,
-                                   *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
+                tmem_ld_32x32b_x32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
+            if (lane == 0) mbar_arrive(bars.s_free);
 
-            float mx = -INFINITY;
+            // row max: eight independent three-input chains, then a short tree
+            float mx8[8];
 #pragma unroll
-            for (int e = 0; e < BT; ++e) mx = fmaxf(mx, __uint_as_float(s[e]));
+            for (int a = 0; a < 8; ++a)
+                mx8[a] = fmaxf(__uint_as_float(s[a]), __uint_as_float(s[a + 8]));
+#pragma unroll
+            for (int e = 16; e < BT; e += 16)
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+                    mx8[a] = fmax3(mx8[a], __uint_as_float(s[e + a]), __uint_as_float(s[e + 8 + a]));
+            const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                                   fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
             const float m_tile = mx * c2;
             bool need;
             float m_use, alpha;
@@ -381,52 +430,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_use = need ? m_new : m_run;
                 alpha = need ? fast_exp2(m_run - m_new) : 1.f;
             }
+            // p = 2^(s*c2 - m): packed fp32x2 scale-and-shift, MUFU exp2, four
+            // independent packed partial sums
             uint32_t pk[BT / 2];
-            float lsum = 0.f;
+            const uint64_t c2x2 = f32x2_pack(c2, c2);
+            const uint64_t negm = f32x2_pack(-m_use, -m_use);
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
             for (int e = 0; e < BT; e += 2) {
-                const float p0 = fast_exp2(fmaf(__uint_as_float(s[e]), c2, -m_use));
-                const float p1 = fast_exp2(fmaf(__uint_as_float(s[e + 1]), c2, -m_use));
-                lsum += p0 + p1;
+                const uint64_t x = f32x2_fma(
+                    f32x2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2x2, negm);
+                float x0, x1;
+                f32x2_unpack(x, x0, x1);
+                const float p0 = fast_exp2(x0);
+                const float p1 = fast_exp2(x1);
+                acc[(e >> 1) & 3] = f32x2_add(acc[(e >> 1) & 3], f32x2_pack(p0, p1));
                 pk[e / 2] = pack_bf16x2(p0, p1);
             }
+            float a0, a1, a2, a3;
+            f32x2_unpack(f32x2_add(acc[0], acc[1]), a0, a1);
+            f32x2_unpack(f32x2_add(acc[2], acc[3]), a2, a3);
+            const float lsum = (a0 + a2) + (a1 + a3);
             l_run = (j == 0) ? lsum : fmaf(l_run, alpha, lsum);
             m_run = m_use;
 
-            if (j > 0) {
-                // P_{j-1} V_{j-1} has finished: the P buffer is free and O is stable.
-                if (!warp_wait_bar(bars.o_done, (j - 1) & 1, p, abort_flag)) {
+            if (__any_sync(0xffffffffu, need)) {
+                // rescale O: P_{j-1} V_{j-1} must have landed first
+                if (!warp_wait_bar(&bars.p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, p, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld_32x32b_x32(tO + cc * 32, o);
-                        tmem_wait_ld();
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(tO + cc * 32, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st_32x32b_x32(tO + cc * 32, o);
-                    }
-                    tmem_wait_st();
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st_32x32b_x32(tO + cc * 32, o);
                 }
             }
-            // P row r -> shared memory, K-major 128-byte-swizzled operand layout.
-#pragma unroll
-            for (int u = 0; u < BT / 8; ++u) {
-                const int c = u >> 3, uc = u & 7;
-                uint4 v = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-                *reinterpret_cast<uint4*>(sP + c * C::kPChunk + r * 128 + ((uc ^ (r & 7)) << 4)) = v;
+            // P_j -> tensor memory buffer j&1, free once P_{j-2} V_{j-2} is done
+            if (j >= 2 && !warp_wait_bar(&bars.p_free[j & 1], ((j - 2) >> 1) & 1, p, abort_flag)) {
+                ok = false;
+                break;
             }
-            fence_proxy_async_smem();
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < BT / 64; ++cc)
+                tmem_st_32x32b_x32(tP + (j & 1) * 64 + cc * 32,
+                                   *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bars.p_full);
+            if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
         }
-        if (ok) ok = warp_wait_bar(bars.o_done, (k - 1) & 1, p, abort_flag);
+        if (ok) ok = warp_wait_bar(&bars.p_free[(k - 1) & 1], ((k - 1) >> 1) & 1, p, abort_flag);
         // every softmax thread gets here (all waits are bounded); the epilogue
         // runs only if all four warps finished their loop
         if (named_barrier_and(1, 128, ok)) {
@@ -571,9 +632,9 @@ veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint1
     prm.k = k;
     prm.scale_log2 = pr.scale * 1.4426950408889634f;
     prm.wait_limit_ns = wait_limit_ns();
-    if (pr.d == 128 && pr.Bt == 128) return launch_cfg<128, 128, 2>(prm, pr, s);
-    if (pr.d == 128 && pr.Bt == 64) return launch_cfg<128, 64, 3>(prm, pr, s);
-    if (pr.d == 64 && pr.Bt == 128) return launch_cfg<64, 128, 3>(prm, pr, s);
+    if (pr.d == 128 && pr.Bt == 128) return launch_cfg<128, 128, 3>(prm, pr, s);
+    if (pr.d == 128 && pr.Bt == 64) return launch_cfg<128, 64, 4>(prm, pr, s);
+    if (pr.d == 64 && pr.Bt == 128) return launch_cfg<64, 128, 4>(prm, pr, s);
     return launch_cfg<64, 64, 4>(prm, pr, s);
 }
 
