@@ -25,11 +25,12 @@
 //                   tensor memory once; then per tile reads S_j from TMEM,
 //                   keeps the running max / sum in fp32 (exp2 with the scale
 //                   folded in, packed fp32x2 arithmetic), writes P_j as bf16
-//                   into one of two TMEM P buffers, and rescales O in TMEM only
+//                   over S_j in tensor memory, and rescales O in TMEM only
 //                   when the running max grows by more than 2^8 (exact: the
 //                   final normalisation uses the same max);
-//   * S_{j+1} is computed while the softmax works on S_j, and P_j V_j runs
-//     while the softmax works on S_{j+1};
+//   * two S/P buffers in tensor memory: the softmax writes P_j over S_j, so it
+//     never waits for the previous P V product, and the tensor core computes
+//     P_{j-1} V_{j-1} and S_{j+1} while the softmax works on tile j;
 //   * the epilogue normalises O, stages it in shared memory and writes it back
 //     with the same 5-D box through a TMA store; lse is written per token.
 // Every wait on an mbarrier is bounded by a time limit; on expiry the CTA sets
@@ -75,15 +76,16 @@ struct Cfg {
     static constexpr int kOffV = kOffK + NS * kKVBytes;
     static constexpr int kOffBar = kOffV + NS * kKVBytes;
     // barriers: q, q_tmem, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS],
-    // s_full, s_free, p_full[2], p_free[2], drain
-    static constexpr int kNumBars = 2 + 4 * NS + 1 + 1 + 2 + 2 + 1;
+    // s_full[2], p_full[2], pv_done[2], drain
+    static constexpr int kNumBars = 2 + 4 * NS + 2 + 2 + 2 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-    // tensor memory columns (all offsets multiples of 64)
-    static constexpr int kTmemS = 0;                 // S_j, fp32, BT columns
-    static constexpr int kTmemP = BT;                // P buffers: 2 x 64 columns of bf16 pairs
-    static constexpr int kTmemQ = BT + 128;          // Q: D/2 columns of bf16 pairs
-    static constexpr int kTmemO = BT + 192;          // O accumulator, fp32, D columns
+    // tensor memory columns (all offsets multiples of 64).  Buffer b holds S_j
+    // (fp32, BT columns) for j = b mod 2, and then P_j (bf16 pairs, the first
+    // BT/2 columns) written over it.
+    static constexpr int kTmemS = 0;                 // S/P buffers 0 and 1
+    static constexpr int kTmemQ = 2 * BT;            // Q: D/2 columns of bf16 pairs
+    static constexpr int kTmemO = 2 * BT + 64;       // O accumulator, fp32, D columns
     static constexpr int kTmemCols = (kTmemO + D) <= 256 ? 256 : 512;
     static_assert(kTmemO + D <= 512, "tensor memory budget");
     static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, BT, false);
@@ -98,9 +100,8 @@ struct Bars {
     uint64_t* k_empty;
     uint64_t* v_empty;
     uint64_t* s_full;
-    uint64_t* s_free;
     uint64_t* p_full;
-    uint64_t* p_free;
+    uint64_t* pv_done;
     uint64_t* drain;
 };
 
@@ -150,18 +151,23 @@ __device__ __forceinline__ void tile_origin(int t, int pt, int ph, int pw, int H
     x0 = (t % nw) * pw;
 }
 
-// Barrier phase bookkeeping (each barrier completes once per use):
+// Barrier phase bookkeeping (each barrier completes once per use; b = j & 1,
+// m = j >> 1):
 //   k_full/v_full[st]   fill n of stage st (tile j = st + n*NS): parity n & 1
 //   k_empty/v_empty[st] the MMA consumed fill n: parity n & 1
-//   s_full              QK_j done: parity j & 1
-//   s_free              softmax has read S_j: parity j & 1
-//   p_full[b]           P_j in TMEM (and O rescaled), j = b + 2m: parity m & 1
-//   p_free[b]           P_j V_j done, j = b + 2m: parity m & 1
+//   s_full[b]           S_j = Q K_j^T is in buffer b: parity m & 1
+//   p_full[b]           P_j has replaced S_j in buffer b (and O is rescaled):
+//                       parity m & 1
+//   pv_done[b]          P_j V_j is done: parity m & 1
 // For every barrier the next completion needs the waiter to have passed its
-// current wait, and no waiter skips a completion it has to see, so a waiter is
-// never two phases away from its barrier and the parities are unambiguous.
-// (P_j V_j completing is read from p_free: the softmax waits on P_{j-2} V_{j-2}
-// in every iteration, which keeps that barrier within one phase.)
+// current wait, so no waiter is two phases behind.  pv_done[b] is waited on
+// only now and then (O rescale, epilogue); it cannot lag by two phases either:
+// when the softmax reaches tile j, S_{j-1} has been computed, and QK_{j-1} was
+// issued after P_{j-3} V_{j-3}, so that product (the previous completion of
+// pv_done[(j-1) & 1]) is done.  Ordering inside the tensor pipe: QK_{j+2}
+// overwrites buffer b after P_j V_j has read P_j from it; both are issued by
+// the same thread in that order, and tcgen05.mma operations issued by one
+// thread execute in issue order.
 template <int D, int BT, int NS>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ AttnParams p) {
@@ -181,10 +187,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars.k_empty = bars.v_full + NS;
     bars.v_empty = bars.k_empty + NS;
     bars.s_full = bars.v_empty + NS;
-    bars.s_free = bars.s_full + 1;
-    bars.p_full = bars.s_free + 1;
-    bars.p_free = bars.p_full + 2;
-    bars.drain = bars.p_free + 2;
+    bars.p_full = bars.s_full + 2;
+    bars.pv_done = bars.p_full + 2;
+    bars.drain = bars.pv_done + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -206,11 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars.k_empty[s], 1);
             mbar_init(&bars.v_empty[s], 1);
         }
-        mbar_init(bars.s_full, 1);
-        mbar_init(bars.s_free, 4);
         for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.s_full[b], 1);
             mbar_init(&bars.p_full[b], 4);
-            mbar_init(&bars.p_free[b], 1);
+            mbar_init(&bars.pv_done[b], 1);
         }
         mbar_init(bars.drain, 1);
         *abort_flag = 0;
@@ -305,49 +309,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ============================================================ MMA issuer
         if (lane == 0) {
             const uint32_t tS = tbase + C::kTmemS;
-            const uint32_t tP = tbase + C::kTmemP;
             const uint32_t tQ = tbase + C::kTmemQ;
             const uint32_t tO = tbase + C::kTmemO;
             const uint32_t k_addr = smem_addr(sK);
             const uint32_t v_addr = smem_addr(sV);
             bool ok = wait_bar(bars.q_tmem, 0, p, abort_flag);
-            // S_j = Q K_j^T: A = Q from tensor memory, B = K tile (K-major, swizzled)
+            // S_j = Q K_j^T into buffer j & 1: A = Q from tensor memory, B = K tile
+            // (K-major, swizzled).  Buffer j & 1 was last read by P_{j-2} V_{j-2},
+            // issued before this by the same thread.
             auto issue_qk = [&](int j) -> bool {
-                const int st = j % NS;
+                const int st = j % NS, b = j & 1;
                 if (!wait_bar(&bars.k_full[st], (j / NS) & 1, p, abort_flag)) return false;
-                if (j >= 1 && !wait_bar(bars.s_free, (j - 1) & 1, p, abort_flag)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const int c = ks >> 2, w = ks & 3;
-                    const uint64_t b = smem_desc_sw128(
+                    const uint64_t bd = smem_desc_sw128(
                         k_addr + st * C::kKVBytes + c * C::kKVChunk + w * 32, 16, 1024);
-                    mma_bf16_ts(tS, tQ + ks * 8, b, C::kIdescQK, ks > 0 ? 1u : 0u);
+                    mma_bf16_ts(tS + b * BT, tQ + ks * 8, bd, C::kIdescQK, ks > 0 ? 1u : 0u);
                 }
-                mma_commit(bars.s_full);
+                mma_commit(&bars.s_full[b]);
                 mma_commit(&bars.k_empty[st]);
                 return true;
             };
             if (ok) ok = issue_qk(0);
+            if (ok && k > 1) ok = issue_qk(1);
             for (int j = 0; j < k && ok; ++j) {
-                if (j + 1 < k && !issue_qk(j + 1)) {
-                    ok = false;
-                    break;
-                }
-                const int st = j % NS;
-                if (!wait_bar(&bars.p_full[j & 1], (j >> 1) & 1, p, abort_flag)) break;
+                const int st = j % NS, b = j & 1;
+                if (!wait_bar(&bars.p_full[b], (j >> 1) & 1, p, abort_flag)) break;
                 if (!wait_bar(&bars.v_full[st], (j / NS) & 1, p, abort_flag)) break;
                 tc_fence_after();
-                // O += P_j V_j: A = P_j from tensor memory, B = V tile (MN-major)
-                const uint32_t pa = tP + (j & 1) * 64;
+                // O += P_j V_j: A = P_j from buffer b, B = V tile (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < BT / 16; ++ks) {
-                    const uint64_t b =
+                    const uint64_t bd =
                         smem_desc_sw128(v_addr + st * C::kKVBytes + ks * 2048, C::kKVChunk, 1024);
-                    mma_bf16_ts(tO, pa + ks * 8, b, C::kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+                    mma_bf16_ts(tO, tS + b * BT + ks * 8, bd, C::kIdescPV,
+                                (j > 0 || ks > 0) ? 1u : 0u);
                 }
-                mma_commit(&bars.p_free[j & 1]);
+                mma_commit(&bars.pv_done[b]);
                 mma_commit(&bars.v_empty[st]);
+                if (j + 2 < k && !issue_qk(j + 2)) break;
             }
             // Drain: all tensor-core work issued by this thread has completed.
             mma_commit(bars.drain);
@@ -360,7 +362,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = wq * 32 + lane;            // query row of the tile
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tbase + lane_off + C::kTmemS;
-        const uint32_t tP = tbase + lane_off + C::kTmemP;
         const uint32_t tQ = tbase + lane_off + C::kTmemQ;
         const uint32_t tO = tbase + lane_off + C::kTmemO;
         const float c2 = p.scale_log2;
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(bars.q_tmem);
         }
         for (int j = 0; j < k && ok; ++j) {
-            if (!warp_wait_bar(bars.s_full, j & 1, p, abort_flag)) {
+            if (!warp_wait_bar(&bars.s_full[j & 1], (j >> 1) & 1, p, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -399,11 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t s[BT];
 #pragma unroll
             for (int cc = 0; cc < BT / 32; ++cc)
-                tmem_ld_32x32b_x32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
+                tmem_ld_32x32b_x32(tS + (j & 1) * BT + cc * 32,
+                                   *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bars.s_free);
 
             // row max: eight independent three-input chains, then a short tree
             float mx8[8];
@@ -456,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             if (__any_sync(0xffffffffu, need)) {
                 // rescale O: P_{j-1} V_{j-1} must have landed first
-                if (!warp_wait_bar(&bars.p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, p, abort_flag)) {
+                if (!warp_wait_bar(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -472,22 +471,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_32x32b_x32(tO + cc * 32, o);
                 }
             }
-            // P_j -> tensor memory buffer j&1, free once P_{j-2} V_{j-2} is done
-            if (j >= 2 && !warp_wait_bar(&bars.p_free[j & 1], ((j - 2) >> 1) & 1, p, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
+            // P_j over S_j in buffer j & 1 (this thread has read its row of S_j)
 #pragma unroll
             for (int cc = 0; cc < BT / 64; ++cc)
-                tmem_st_32x32b_x32(tP + (j & 1) * 64 + cc * 32,
+                tmem_st_32x32b_x32(tS + (j & 1) * BT + cc * 32,
                                    *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
         }
-        if (ok) ok = warp_wait_bar(&bars.p_free[(k - 1) & 1], ((k - 1) >> 1) & 1, p, abort_flag);
+        if (ok) ok = warp_wait_bar(&bars.pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, p, abort_flag);
         // every softmax thread gets here (all waits are bounded); the epilogue
         // runs only if all four warps finished their loop
         if (named_barrier_and(1, 128, ok)) {
