@@ -134,6 +134,18 @@ def test_sparse_attn_dims_and_tile_sizes(vb, oracle, d, shape):
     _attn_case(vb, oracle, w, t, idx, None)
 
 
+@pytest.mark.parametrize("d,shape,grid", [(128, (1, 8, 16), (3, 8, 16)), (64, (1, 8, 8), (5, 8, 8))])
+def test_odd_tile_count(vb, oracle, d, shape, grid):
+    """nT odd: the last CTA owns a single query tile."""
+    w = workloads.custom("odd", 1, 2, d, grid, [shape], 2)
+    assert w.nT % 2 == 1
+    t = _inputs(w, "cuda")
+    rng = np.random.default_rng(11)
+    idx = np.stack([rng.permutation(w.nT)[:w.k] for _ in range(w.H * w.nT)])
+    idx = idx.reshape(1, w.H, w.nT, w.k).astype(np.int32)
+    _attn_case(vb, oracle, w, t, idx, None)
+
+
 def test_k_equals_all_tiles_is_dense_path(vb, oracle):
     """k = nT through an index list equals the dense schedule bit for bit, and the oracle."""
     w = workloads.custom("dense", 1, 2, 128, (4, 16, 32), [(2, 8, 8)], 16)

@@ -48,6 +48,10 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kSoftmaxWarp0 = 4;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+#ifndef VEDA_POLY_PAIRS
+#define VEDA_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = VEDA_POLY_PAIRS;  // of every 8 exp2 pairs, on the FMA pipe
 
 struct __align__(64) AttnParams {
     CUtensorMap tmQ[kMaxShapes];
@@ -75,9 +79,9 @@ struct Cfg {
     static constexpr int kOffK = kQBytes;
     static constexpr int kOffV = kOffK + NS * kKVBytes;
     static constexpr int kOffBar = kOffV + NS * kKVBytes;
-    // barriers: q, q_tmem, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS],
-    // s_full[2], p_full[2], pv_done[2], drain
-    static constexpr int kNumBars = 2 + 4 * NS + 2 + 2 + 2 + 1;
+    // barriers: q, q_tmem, k_full[NS], v_full[NS], kv_empty[NS], s_full[2],
+    // p_full[2], drain
+    static constexpr int kNumBars = 2 + 3 * NS + 2 + 2 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     // tensor memory columns (all offsets multiples of 64).  Buffer b holds S_j
@@ -97,11 +101,9 @@ struct Bars {
     uint64_t* q_tmem;
     uint64_t* k_full;
     uint64_t* v_full;
-    uint64_t* k_empty;
-    uint64_t* v_empty;
+    uint64_t* kv_empty;
     uint64_t* s_full;
     uint64_t* p_full;
-    uint64_t* pv_done;
     uint64_t* drain;
 };
 
@@ -152,19 +154,20 @@ __device__ __forceinline__ void tile_origin(int t, int pt, int ph, int pw, int H
 }
 
 // Barrier phase bookkeeping (each barrier completes once per use; b = j & 1,
-// m = j >> 1):
-//   k_full/v_full[st]   fill n of stage st (tile j = st + n*NS): parity n & 1
-//   k_empty/v_empty[st] the MMA consumed fill n: parity n & 1
+// m = j >> 1; stage st = j % NS holds K_j and V_j, fill n = j / NS):
+//   k_full/v_full[st]   fill n of stage st has landed: parity n & 1
+//   kv_empty[st]        P_j V_j is done, so K_j and V_j are consumed (one
+//                       commit per tile): parity n & 1
 //   s_full[b]           S_j = Q K_j^T is in buffer b: parity m & 1
 //   p_full[b]           P_j has replaced S_j in buffer b (and O is rescaled):
 //                       parity m & 1
-//   pv_done[b]          P_j V_j is done: parity m & 1
 // For every barrier the next completion needs the waiter to have passed its
-// current wait, so no waiter is two phases behind.  pv_done[b] is waited on
-// only now and then (O rescale, epilogue); it cannot lag by two phases either:
-// when the softmax reaches tile j, S_{j-1} has been computed, and QK_{j-1} was
-// issued after P_{j-3} V_{j-3}, so that product (the previous completion of
-// pv_done[(j-1) & 1]) is done.  Ordering inside the tensor pipe: QK_{j+2}
+// current wait, so no waiter is two phases behind.  The softmax reads
+// "P_{j-1} V_{j-1} done" from kv_empty only now and then (O rescale,
+// epilogue); it cannot trail that barrier by two phases either: when S_j is
+// visible, QK_j and everything issued before it (P_{j-2} V_{j-2} and older) is
+// done, so the previous completion of that stage is.  The next one needs
+// P_{j+NS-1}, which needs the softmax to have finished tile j.  Ordering inside the tensor pipe: QK_{j+2}
 // overwrites buffer b after P_j V_j has read P_j from it; both are issued by
 // the same thread in that order, and tcgen05.mma operations issued by one
 // thread execute in issue order.
@@ -184,12 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars.q_tmem = bar_base + 1;
     bars.k_full = bar_base + 2;
     bars.v_full = bars.k_full + NS;
-    bars.k_empty = bars.v_full + NS;
-    bars.v_empty = bars.k_empty + NS;
-    bars.s_full = bars.v_empty + NS;
+    bars.kv_empty = bars.v_full + NS;
+    bars.s_full = bars.kv_empty + NS;
     bars.p_full = bars.s_full + 2;
-    bars.pv_done = bars.p_full + 2;
-    bars.drain = bars.pv_done + 2;
+    bars.drain = bars.p_full + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -208,13 +209,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < NS; ++s) {
             mbar_init(&bars.k_full[s], 1);
             mbar_init(&bars.v_full[s], 1);
-            mbar_init(&bars.k_empty[s], 1);
-            mbar_init(&bars.v_empty[s], 1);
+            mbar_init(&bars.kv_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.s_full[b], 1);
             mbar_init(&bars.p_full[b], 4);
-            mbar_init(&bars.pv_done[b], 1);
         }
         mbar_init(bars.drain, 1);
         *abort_flag = 0;
@@ -270,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int j = j0 + jj, st = j % NS, n = j / NS;
                     int t0, y0, x0;
                     tile_origin(t, pt, ph, pw, p.Hs, p.Ws, t0, y0, x0);
-                    if (n > 0) good = wait_bar(&bars.k_empty[st], (n - 1) & 1, p, abort_flag);
+                    if (n > 0) good = wait_bar(&bars.kv_empty[st], (n - 1) & 1, p, abort_flag);
                     if (good) {
                         mbar_arrive_expect_tx(&bars.k_full[st], C::kKVBytes);
 #pragma unroll
@@ -278,8 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_5d(sK + st * C::kKVBytes + c * C::kKVChunk, &p.tmK[slot],
                                         &bars.k_full[st], c * 64, x0, y0, t0, bh);
                         k_fills = j + 1;
-                        if (n > 0) good = wait_bar(&bars.v_empty[st], (n - 1) & 1, p, abort_flag);
-                        if (good) {
+                        {
                             mbar_arrive_expect_tx(&bars.v_full[st], C::kKVBytes);
 #pragma unroll
                             for (int c = 0; c < C::kChunks; ++c)
@@ -329,7 +327,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_bf16_ts(tS + b * BT, tQ + ks * 8, bd, C::kIdescQK, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(&bars.s_full[b]);
-                mma_commit(&bars.k_empty[st]);
                 return true;
             };
             if (ok) ok = issue_qk(0);
@@ -347,8 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_bf16_ts(tO, tS + b * BT + ks * 8, bd, C::kIdescPV,
                                 (j > 0 || ks > 0) ? 1u : 0u);
                 }
-                mma_commit(&bars.pv_done[b]);
-                mma_commit(&bars.v_empty[st]);
+                mma_commit(&bars.kv_empty[st]);
                 if (j + 2 < k && !issue_qk(j + 2)) break;
             }
             // Drain: all tensor-core work issued by this thread has completed.
@@ -429,8 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_use = need ? m_new : m_run;
                 alpha = need ? fast_exp2(m_run - m_new) : 1.f;
             }
-            // p = 2^(s*c2 - m): packed fp32x2 scale-and-shift, MUFU exp2, four
-            // independent packed partial sums
+            // p = 2^(s*c2 - m): packed fp32x2 scale-and-shift; kPolyPairs of
+            // every 8 element pairs take the FMA-pipe exp2, the others MUFU
+            // ex2 (the two units then share the load); four independent packed
+            // partial sums
             uint32_t pk[BT / 2];
             const uint64_t c2x2 = f32x2_pack(c2, c2);
             const uint64_t negm = f32x2_pack(-m_use, -m_use);
@@ -439,10 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < BT; e += 2) {
                 const uint64_t x = f32x2_fma(
                     f32x2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2x2, negm);
-                float x0, x1;
-                f32x2_unpack(x, x0, x1);
-                const float p0 = fast_exp2(x0);
-                const float p1 = fast_exp2(x1);
+                float p0, p1;
+                if (((e >> 1) & 7) < kPolyPairs) {
+                    f32x2_unpack(exp2_poly_x2(x), p0, p1);
+                } else {
+                    float x0, x1;
+                    f32x2_unpack(x, x0, x1);
+                    p0 = fast_exp2(x0);
+                    p1 = fast_exp2(x1);
+                }
                 acc[(e >> 1) & 3] = f32x2_add(acc[(e >> 1) & 3], f32x2_pack(p0, p1));
                 pk[e / 2] = pack_bf16x2(p0, p1);
             }
@@ -455,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             if (__any_sync(0xffffffffu, need)) {
                 // rescale O: P_{j-1} V_{j-1} must have landed first
-                if (!warp_wait_bar(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p, abort_flag)) {
+                if (!warp_wait_bar(&bars.kv_empty[(j - 1) % NS], ((j - 1) / NS) & 1, p, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -481,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
         }
-        if (ok) ok = warp_wait_bar(&bars.pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, p, abort_flag);
+        if (ok) ok = warp_wait_bar(&bars.kv_empty[(k - 1) % NS], ((k - 1) / NS) & 1, p, abort_flag);
         // every softmax thread gets here (all waits are bounded); the epilogue
         // runs only if all four warps finished their loop
         if (named_barrier_and(1, 128, ok)) {
