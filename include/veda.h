@@ -102,8 +102,11 @@ veda_status veda_tripool(const veda_problem* p, const uint16_t* Q, const uint16_
  *   Wq, Wk: fp32 [H, d, d] (row = input channel, column = output channel)
  *   S     : fp32 [B, H, nT, nT]
  *   ws    : device workspace of at least
- *           VEDA_STATUS_BYTES + 2 * B*H*nT*3*d*4 bytes (projected statistics).
- * Arithmetic is fp32.
+ *           VEDA_STATUS_BYTES + 2 * B*H*nT*9*d*4 bytes (projected statistics,
+ *           stored as TF32 hi/lo splits).
+ * The projection is fp32; the score is a tensor-core product of three TF32
+ * terms (hi.hi + hi.lo + lo.hi, fp32 accumulation), within about 3 * 2^-21 of
+ * the fp32 product per term.
  */
 veda_status veda_tile_score(const veda_problem* p, const float* statsQ, const float* statsK,
                             const float* Wq, const float* Wk, float* S, void* ws,
@@ -171,7 +174,7 @@ veda_status veda_get_status(const void* ws, veda_stream_t stream, int32_t* devic
  * array inside the library instead of a caller workspace:
  *   - the array holds veda_noalloc_scratch_bytes() bytes (64 MiB); every GPU
  *     that loads the library keeps it until the process exits;
- *   - a problem needing more than VEDA_STATUS_BYTES + 2*B*H*nT*3*d*4 bytes of
+ *   - a problem needing more than VEDA_STATUS_BYTES + 2*B*H*nT*9*d*4 bytes of
  *     it returns VEDA_ERR_UNSUPPORTED and launches nothing;
  *   - the first call on a device looks up the array's address on that device
  *     (the device must be current); make that first call before any stream

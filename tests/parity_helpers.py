@@ -5,8 +5,10 @@ Parity rules (tolerances derived from the arithmetic):
 * TripPool max/min: bit-exact (a max of bf16 values is exact in fp32);
   avg: |gpu - oracle| <= (Bt - 1) * 2^-24 * mean|x| + 2^-24 * |avg|, the error
   bound of an fp32 sum of Bt terms followed by an exact division by 2^m.
-* scores: |gpu - oracle| <= 4e-5 * (|stats_q| |W_q|) . (|stats_k| |W_k|)^T, the
-  fp32 dot-product bound (d + 3d + 4) * 2^-24 <= 3.1e-5 on the absolute terms.
+* scores: |gpu - oracle| <= 8e-5 * (|stats_q| |W_q|) . (|stats_k| |W_k|)^T: the
+  fp32 projection (d terms), the three-term TF32 product (<= 3 * 2^-21 per term)
+  and fp32 accumulation of 9d products: (d + 9d + 4) * 2^-24 + 3 * 2^-21 <= 7.8e-5
+  on the absolute terms.
 * mask rows: bit-exact wherever the oracle's k-th and (k+1)-th scores differ
   by more than 1e-3 relative; in other rows the GPU row must hold exactly k
   tiles and every tile whose oracle score clears s_(k) by that margin.
@@ -25,7 +27,7 @@ from oracle import Oracle
 O_MAX_ABS = 2e-2
 O_MEAN_ABS = 5e-3
 LSE_ABS = 2e-3
-SCORE_GAMMA = 4e-5
+SCORE_GAMMA = 8e-5
 GAP_REL = 1e-3
 
 

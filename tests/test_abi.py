@@ -87,8 +87,9 @@ def test_workspace_size_matches_layout(lib):
     prob = _problem(vb, B=2, H=3, tile_shapes=[(2, 8, 8)], k=5)
     nT, d = 16, 128
     stats = 2 * 3 * nT * 3 * d * 4
+    proj = 2 * 3 * nT * 9 * d * 4
     S = 2 * 3 * nT * nT * 4
     idx = 2 * 3 * nT * 5 * 4
     r256 = lambda x: (x + 255) // 256 * 256
-    want = 256 + 4 * r256(stats) + r256(S) + r256(idx)
+    want = 256 + 2 * r256(proj) + 2 * r256(stats) + r256(S) + r256(idx)
     assert vb.veda_workspace_size(prob) == want

@@ -38,10 +38,17 @@ veda_status cuda_check(cudaError_t err, const char* what);
 // error after checking the launch.
 veda_status launch_tripool(const Problem& pr, const uint16_t* Q, const uint16_t* K, float* statsQ,
                            float* statsK, cudaStream_t s);
+// Projection of statsQ (side 0) or statsK (side 1) into the TF32-split score
+// operand layout [B*H*nT][9d] (see tile_score.cu).
 veda_status launch_project(const Problem& pr, const float* stats, const float* W, float* out,
-                           cudaStream_t s);
-veda_status launch_score(const Problem& pr, const float* qt, const float* kt, float* S,
-                         cudaStream_t s);
+                           int side, cudaStream_t s);
+// S = q^ k^^T on the tensor cores (score_tc.cu); status: device status word.
+veda_status launch_score(const Problem& pr, const float* qext, const float* kext, float* S,
+                         int* status, cudaStream_t s);
+// Bytes of one projected-statistics operand: B*H*nT*9d fp32.
+inline size_t projected_bytes(const Problem& pr) {
+    return (size_t)pr.B * pr.H * pr.nT * 9 * pr.d * sizeof(float);
+}
 veda_status launch_topk(const Problem& pr, const float* S, uint8_t* mask, int32_t* idx,
                         cudaStream_t s);
 veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint16_t* K,

@@ -75,8 +75,8 @@ veda_status veda_tile_score_noalloc(const veda_problem* p, const float* statsQ,
         (st = veda::check_ptr(Wq, "Wq")) || (st = veda::check_ptr(Wk, "Wk")) ||
         (st = veda::check_ptr(S, "S")))
         return st;
-    // Same scratch layout as veda_tile_score's workspace: status word, q~, k~.
-    const size_t stats = (size_t)pr.B * pr.H * pr.nT * 3 * pr.d * sizeof(float);
+    // Same scratch layout as veda_tile_score's workspace: status word, q^, k^.
+    const size_t stats = veda::projected_bytes(pr);
     const size_t need = VEDA_STATUS_BYTES + 2 * stats;
     if (need > kVedaNoallocScratchBytes)
         return veda::fail(VEDA_ERR_UNSUPPORTED,
@@ -92,9 +92,9 @@ veda_status veda_tile_score_noalloc(const veda_problem* p, const float* statsQ,
     float* kt = reinterpret_cast<float*>(base + VEDA_STATUS_BYTES + stats);
     if ((st = veda::cuda_check(cudaMemsetAsync(base, 0, VEDA_STATUS_BYTES, s), "status reset")))
         return st;
-    if ((st = veda::launch_project(pr, statsQ, Wq, qt, s))) return st;
-    if ((st = veda::launch_project(pr, statsK, Wk, kt, s))) return st;
-    return veda::launch_score(pr, qt, kt, S, s);
+    if ((st = veda::launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
+    if ((st = veda::launch_project(pr, statsK, Wk, kt, 1, s))) return st;
+    return veda::launch_score(pr, qt, kt, S, reinterpret_cast<int*>(base), s);
 }
 
 }  // extern "C"

@@ -1,0 +1,255 @@
+// score_tc.cu -- the tile-pair score matrix on the tensor cores.
+//
+// "Veda: Scalable Video Diffusion via Distilled Sparse Attention" (project
+// page), "Attention Structure Distillation", Estimator:
+//   S[i, j] = sum over s in {avg, max, min} of <q~_{i,s}, k~_{j,s}>,
+// an nT x nT x 3d contraction per head.
+//
+// The decision that follows (Top-k) wants fp32-grade scores, so the product
+// runs as a three-term TF32 split: every fp32 value x is written by the
+// projection as hi = x rounded to TF32 and lo = x - hi, with
+//   q^ = [q_hi | q_hi | q_lo],  k^ = [k_hi | k_lo | k_hi]   (length 9d),
+// so that q^ . k^ = q_hi k_hi + q_hi k_lo + q_lo k_hi, which differs from the
+// fp32 product by at most about 3 * 2^-21 |q||k| per term (the dropped lo*lo
+// term and the TF32 truncation of lo); accumulation is fp32 in tensor memory.
+// S = q^ k^^T is then one kind::tf32 GEMM with K = 9d:
+//   * one CTA per 128 x 128 block of S of one head; 128 threads;
+//   * warp 0 lane 0 streams 32-wide K blocks of q^ and k^ (128 rows x 128 B,
+//     128-byte swizzle) by TMA into a 3-stage ring;
+//   * warp 1 allocates 128 TMEM columns; its lane 0 issues 4 tcgen05.mma
+//     (M = N = 128, K = 8) per K block;
+//   * all four warps read the accumulator back (thread = row) and store S.
+// Waits are bounded (VEDA_ERR_TIMEOUT in the status word, then a bounded drain
+// of the copies and products in flight before tensor memory is freed).
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace veda {
+
+namespace {
+
+constexpr int kScoreThreads = 128;
+constexpr int kStages = 3;
+constexpr int kTileBytes = 128 * 128;             // 128 rows x 32 fp32
+constexpr int kStageBytes = 2 * kTileBytes;       // A and B
+constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
+// kind::tf32, fp32 accumulate, both operands K-major, M = N = 128
+constexpr uint32_t kIdescTF32 = (1u << 4) | (2u << 7) | (2u << 10) | ((128u >> 3) << 17) |
+                                ((128u >> 4) << 24);
+
+struct __align__(64) ScoreParams {
+    CUtensorMap mapA;  // q^: rows B*H*nT, K = 9d
+    CUtensorMap mapB;  // k^
+    float* S;
+    int* status;
+    int nT, kblocks;
+    unsigned long long wait_limit_ns;
+};
+
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// Bounded wait (suspending in hardware between tests); false on expiry.
+__device__ __forceinline__ bool wait_limited(uint64_t* bar, uint32_t parity,
+                                             const ScoreParams& p) {
+    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait_sleep(bar, parity, 20000)) {
+        if (global_timer_ns() - t0 > p.wait_limit_ns) {
+            atomicCAS(p.status, 0, (int)VEDA_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kScoreThreads, 1)
+    score_tc_kernel(const __grid_constant__ ScoreParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* done = empty + kStages;
+    uint64_t* drain = done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j0 = blockIdx.x * 128, i0 = blockIdx.y * 128, bh = blockIdx.z;
+    const int rowA = bh * p.nT + i0, rowB = bh * p.nT + j0;
+    const int KB = p.kblocks;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    bool ok = true;
+    if (warp == 0 && lane == 0) {
+        // ---------------------------------------------------------- producer
+        tma_prefetch_desc(&p.mapA);
+        tma_prefetch_desc(&p.mapB);
+        int issued = 0;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int st = kb % kStages, n = kb / kStages;
+            if (n > 0 && !wait_limited(&empty[st], (n - 1) & 1, p)) break;
+            uint8_t* a = smem + st * kStageBytes;
+            mbar_arrive_expect_tx(&full[st], kStageBytes);
+            tma_load_2d(a, &p.mapA, &full[st], kb * 32, rowA);
+            tma_load_2d(a + kTileBytes, &p.mapB, &full[st], kb * 32, rowB);
+            issued = kb + 1;
+        }
+        for (int st = 0; st < kStages; ++st)  // drain: the last fill of every stage
+            if (st < issued) wait_limited(&full[st], ((issued - 1 - st) / kStages) & 1, p);
+    } else if (warp == 1 && lane == 0) {
+        // ---------------------------------------------------------- MMA issuer
+        const uint32_t base = smem_addr(smem);
+        for (int kb = 0; kb < KB && ok; ++kb) {
+            const int st = kb % kStages;
+            if (!wait_limited(&full[st], (kb / kStages) & 1, p)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a = base + st * kStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = smem_desc_sw128(a + kk * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(a + kTileBytes + kk * 32, 16, 1024);
+                mma_tf32_ss(tbase, ad, bd, kIdescTF32, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[st]);
+        }
+        mma_commit(done);
+        mma_commit(drain);
+        wait_limited(drain, 0, p);
+    }
+    __syncwarp();
+
+    // -------------------------------------------------------------- epilogue
+    int got = 0;
+    if (lane == 0) got = wait_limited(done, 0, p) ? 1 : 0;
+    got = __shfl_sync(0xffffffffu, got, 0);
+    __syncwarp();
+    if (got) {
+        tc_fence_after();
+        const int r = warp * 32 + lane;
+        const int i = i0 + r;
+        const uint32_t taddr = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+        float* srow = p.S + ((size_t)bh * p.nT + i) * p.nT;
+        const bool vec = (p.nT % 4) == 0;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(taddr + cc * 32, v);
+            tmem_wait_ld();
+            const int jb = j0 + cc * 32;
+            if (i < p.nT) {
+                if (vec && jb + 32 <= p.nT) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(srow + jb + e) =
+                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (jb + e < p.nT) srow[jb + e] = __uint_as_float(v[e]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 128);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows, int kext) {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    if (fn == nullptr) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[2] = {(cuuint64_t)kext, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kext * 4};
+    const cuuint32_t box[2] = {32, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled (score) failed: " + std::to_string((int)r));
+    return VEDA_OK;
+}
+
+}  // namespace
+
+veda_status launch_score(const Problem& pr, const float* qext, const float* kext, float* S,
+                         int* status, cudaStream_t s) {
+    ScoreParams prm;
+    memset(&prm, 0, sizeof(prm));
+    const long long rows = (long long)pr.B * pr.H * pr.nT;
+    const int kx = 9 * pr.d;
+    veda_status st;
+    if ((st = encode_rows_map(&prm.mapA, qext, rows, kx)) != VEDA_OK) return st;
+    if ((st = encode_rows_map(&prm.mapB, kext, rows, kx)) != VEDA_OK) return st;
+    prm.S = S;
+    prm.status = status;
+    prm.nT = pr.nT;
+    prm.kblocks = kx / 32;
+    const char* env = getenv("VEDA_WAIT_LIMIT_MS");
+    unsigned long long ms = 10000ull;
+    if (env != nullptr && atoll(env) > 0) ms = (unsigned long long)atoll(env);
+    prm.wait_limit_ns = ms * 1000000ull;
+    cudaError_t err = cudaFuncSetAttribute(score_tc_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return cuda_check(err, "score smem attribute");
+    const int tiles = (pr.nT + 127) / 128;
+    dim3 grid(tiles, tiles, pr.B * pr.H);
+    score_tc_kernel<<<grid, kScoreThreads, kSmemBytes, s>>>(prm);
+    return cuda_check(cudaGetLastError(), "score launch");
+}
+
+}  // namespace veda

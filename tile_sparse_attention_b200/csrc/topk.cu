@@ -7,9 +7,10 @@
 // go to the lower tile index; -0.0 and +0.0 tie.
 //
 // One warp per row.  Scores become order-preserving 32-bit keys (larger score
-// -> larger key), held in shared memory.  An exact 4-pass radix select
-// (8 bits per pass, most significant first) finds the k-th largest key K* and
-// how many keys equal to K* are kept (the lowest-index ones).  A final pass in
+// -> larger key), held in shared memory.  An exact radix select (8 bits per
+// pass, most significant first, over the bits in which the row's keys differ)
+// finds the k-th largest key K* and how many keys equal to K* are kept (the
+// lowest-index ones).  A final pass in
 // ascending index order emits the mask and, through warp ballots and prefix
 // pop-counts, the index list already sorted.  The selection is an integer
 // computation on the fp32 scores, so it is exactly reproducible.
@@ -47,16 +48,32 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(const __grid_constant_
 
     for (int j = lane; j < nT; j += 32) keys[j] = order_key(__ldg(srow + j));
 
-    uint32_t prefix = 0, pmask = 0;
+    // Bits above the highest bit in which the row's keys differ are common to
+    // all keys: the radix passes start below them, so the first histogram is
+    // spread out instead of piling every key into one bin.
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j = lane; j < nT; j += 32) {
+        kmin = min(kmin, keys[j]);
+        kmax = max(kmax, keys[j]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+    }
+    const int top = 32 - __clz(kmin ^ kmax);  // number of bits that vary (0..32)
+    uint32_t prefix = kmin & (top == 32 ? 0u : ~((1u << top) - 1u));
+    uint32_t pmask = top == 32 ? 0u : ~((1u << top) - 1u);
     int kr = p.k;  // rank of the wanted key among the candidates, from the top
 #pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
+    for (int hi = top; hi > 0; hi -= 8) {
+        const int shift = hi >= 8 ? hi - 8 : 0;
+        const uint32_t dmask = (hi >= 8 ? 255u : (1u << hi) - 1u);
         for (int b = lane; b < 256; b += 32) hist[b] = 0;
         __syncwarp();
         for (int j = lane; j < nT; j += 32) {
             const uint32_t key = keys[j];
-            if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
         }
         __syncwarp();
         // lane l owns bins 255-8l ... 248-8l (descending digit order)
@@ -92,7 +109,7 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(const __grid_constant_
         above = __shfl_sync(0xffffffffu, above, src);
         kr -= (int)above;
         prefix |= digit << shift;
-        pmask |= 255u << shift;
+        pmask |= dmask << shift;
         __syncwarp();
     }
     const uint32_t thr = prefix;  // k-th largest key; keep kr of the keys equal to it

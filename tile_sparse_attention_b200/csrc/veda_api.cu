@@ -103,13 +103,14 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 WorkspaceLayout workspace_layout(const Problem& pr) {
     WorkspaceLayout w{};
     const size_t stats = (size_t)pr.B * pr.H * pr.nT * 3 * pr.d * sizeof(float);
+    const size_t proj = projected_bytes(pr);
     size_t off = 0;
     w.status = off;
     off += VEDA_STATUS_BYTES;
     w.qt = off;  // tile_score's own workspace follows the status word
-    off = align256(off + stats);
+    off = align256(off + proj);
     w.kt = off;
-    off = align256(off + stats);
+    off = align256(off + proj);
     w.statsQ = off;
     off = align256(off + stats);
     w.statsK = off;
@@ -169,9 +170,9 @@ veda_status veda_tile_score(const veda_problem* p, const float* statsQ, const fl
     float* kt = reinterpret_cast<float*>(base + w.kt);
     if ((st = cuda_check(cudaMemsetAsync(base + w.status, 0, sizeof(int), s), "status reset")))
         return st;
-    if ((st = launch_project(pr, statsQ, Wq, qt, s))) return st;
-    if ((st = launch_project(pr, statsK, Wk, kt, s))) return st;
-    return launch_score(pr, qt, kt, S, s);
+    if ((st = launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
+    if ((st = launch_project(pr, statsK, Wk, kt, 1, s))) return st;
+    return launch_score(pr, qt, kt, S, reinterpret_cast<int*>(base + w.status), s);
 }
 
 veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask, int32_t* idx,
@@ -226,9 +227,9 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
     if ((st = cuda_check(cudaMemsetAsync(status, 0, sizeof(int), s), "status reset"))) return st;
     if ((st = launch_tripool(pr, Q, K, statsQ, statsK, s))) return st;
-    if ((st = launch_project(pr, statsQ, Wq, qt, s))) return st;
-    if ((st = launch_project(pr, statsK, Wk, kt, s))) return st;
-    if ((st = launch_score(pr, qt, kt, S, s))) return st;
+    if ((st = launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
+    if ((st = launch_project(pr, statsK, Wk, kt, 1, s))) return st;
+    if ((st = launch_score(pr, qt, kt, S, status, s))) return st;
     if ((st = launch_topk(pr, S, mask_out, idx, s))) return st;
     return launch_sparse_attn(pr, Q, K, V, idx, pr.k, O, lse, status, s);
 }
