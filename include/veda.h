@@ -157,6 +157,36 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
                          veda_stream_t stream);
 
 /*
+ * Max-pooled full-attention teacher (project page, "Attention Structure
+ * Distillation", Teacher; "Empirical Study" 02, Controlled Mask Intervention):
+ *   teacher[b,h,i,j] = max over query tokens q of tile i and key tokens of
+ *                      tile j of P[q, key],  P = softmax(scale * q.k) over all N keys.
+ * Runs the dense attention schedule (every key tile) first, which also yields
+ *   O_dense  : bf16 [B, H, N, d], dense attention output
+ *   lse_dense: fp32 [B, H, N], ln of each row's softmax normaliser
+ * and then one Q K^T pass per tile pair that max-pools exp(scale*s - lse).
+ *   teacher: fp32 [B, H, nT, nT] (k is not used)
+ *   ws     : at least VEDA_STATUS_BYTES bytes
+ * The oracle mask of the page is veda_topk_mask applied to `teacher`.
+ */
+veda_status veda_teacher(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
+                         const uint16_t* V, uint16_t* O_dense, float* lse_dense, float* teacher,
+                         void* ws, veda_stream_t stream);
+
+/*
+ * Tile recall (project page, "Empirical Study" 02): the fraction of the
+ * reference mask's tiles that a predicted mask also selects.
+ *   idx_pred, idx_ref: int32 [B, H, nT, k], each row ascending and duplicate-free
+ *   recall_rows: fp32 [B, H, nT] per-row recall, or NULL
+ *   recall_mean: one fp64 on the device, hits / (B*H*nT*k)
+ *   ws         : at least VEDA_STATUS_BYTES bytes (holds the hit counter)
+ * Integer counting: exact and deterministic.
+ */
+veda_status veda_tile_recall(const veda_problem* p, const int32_t* idx_pred,
+                             const int32_t* idx_ref, float* recall_rows, double* recall_mean,
+                             void* ws, veda_stream_t stream);
+
+/*
  * Waits for `stream`, then copies the device status word of `ws` into
  * *device_status (VEDA_OK or a device-detected veda_status code).
  */

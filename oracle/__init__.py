@@ -56,6 +56,8 @@ def _bind(lib):
     lib.oracle_sparse_attention.argtypes = ([_I64] * 6 + [_P, _I64, ctypes.c_double]
                                             + [_P] * 4 + [_I64, _P, _P, _P])
     lib.oracle_teacher.argtypes = [_I64] * 6 + [_P, ctypes.c_double, _P, _P, _P, _P]
+    lib.oracle_tile_recall.argtypes = [_I64, _I64, _P, _P, _P]
+    lib.oracle_tile_recall.restype = ctypes.c_double
     return lib
 
 
@@ -195,3 +197,13 @@ class Oracle:
         self.lib.oracle_teacher(B, H, d, T, Hs, Ws, _ptr(s), float(scale), _ptr(Q), _ptr(K),
                                 _ptr(teacher), _ptr(lse))
         return teacher, lse
+
+    def tile_recall(self, idx_pred, idx_ref):
+        """Per-row recall of idx_ref by idx_pred (same shape [..., k]) and the mean."""
+        a = np.ascontiguousarray(idx_pred, dtype=np.int32)
+        b = np.ascontiguousarray(idx_ref, dtype=np.int32)
+        k = a.shape[-1]
+        rows = a.size // k
+        per = np.empty(a.shape[:-1], dtype=np.float64)
+        mean = self.lib.oracle_tile_recall(rows, k, _ptr(a), _ptr(b), _ptr(per))
+        return per, float(mean)

@@ -360,3 +360,27 @@ void oracle_teacher(int64_t B, int64_t H, int64_t d, int64_t T, int64_t Hs, int6
         free(key_tile);
     }
 }
+
+/*
+ * Tile recall (Empirical Study 02, "Controlled Mask Intervention": the share
+ * of oracle-selected tiles that a predicted mask recovers).  Per row, the
+ * number of reference tiles that also appear in the predicted row, divided by
+ * k; returns the mean over rows.
+ *   pred, ref: [rows, k] tile indices;  per_row: [rows] (may be NULL)
+ */
+double oracle_tile_recall(int64_t rows, int64_t k, const int32_t* pred, const int32_t* ref,
+                          double* per_row) {
+    double total = 0.0;
+    for (int64_t row = 0; row < rows; ++row) {
+        int64_t hits = 0;
+        for (int64_t a = 0; a < k; ++a) {
+            int found = 0;
+            for (int64_t b = 0; b < k; ++b)
+                if (pred[row * k + b] == ref[row * k + a]) found = 1;
+            hits += found;
+        }
+        if (per_row) per_row[row] = (double)hits / (double)k;
+        total += (double)hits;
+    }
+    return total / ((double)rows * (double)k);
+}

@@ -1,0 +1,110 @@
+"""GPU parity of the training-side tile metrics: the max-pooled full-attention
+teacher, the oracle mask (Top-k of the teacher) and tile recall.
+
+Project page, "Attention Structure Distillation" (Teacher) and "Empirical
+Study" 02 (Controlled Mask Intervention: oracle mask, tile recall).
+
+Teacher tolerance: T = exp(scale * max s - lse); the GPU's s is an fp32 sum of
+d exact bf16 products (error <= d * 2^-24 * sum|q_c k_c|, about 1e-3 here) and
+lse comes from the dense pass (fp32), so |T_gpu / T_oracle - 1| stays below
+about 1e-4; the test allows 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import parity_helpers as ph
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def vb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import tile_sparse_attention_b200 as m
+    m.load_library()
+    return m
+
+
+def _run_teacher(vb, w, t):
+    prob = vb.Problem.from_workload(w)
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    T = torch.empty((w.B, w.H, w.nT, w.nT), dtype=torch.float32, device="cuda")
+    ws = vb.alloc_workspace(prob)
+    vb.veda_teacher(prob, t["Q"], t["K"], t["V"], O, lse, T, ws)
+    assert vb.veda_get_status(ws) == 0
+    return T, lse, O
+
+
+CASES = [
+    ("tiny", lambda: workloads.tiny()),
+    ("mixed", lambda: workloads.custom("mixed", 1, 3, 128, (4, 16, 32),
+                                       [(1, 8, 16), (2, 8, 8), (4, 4, 8)], 3)),
+    ("d64_bt128", lambda: workloads.custom("d64", 1, 2, 64, (4, 16, 32), [(2, 8, 8)], 4)),
+]
+
+
+@pytest.mark.parametrize("name,make", CASES)
+def test_teacher_and_oracle_mask(vb, oracle, name, make):
+    w = make()
+    t = {n: v.cuda() for n, v in workloads.generate(w, device="cpu").items()}
+    T, lse, _ = _run_teacher(vb, w, t)
+    Qb, Kb = ph.to_host_bits(t["Q"]), ph.to_host_bits(t["K"])
+    T_o, lse_o = oracle.teacher(Qb, Kb, w.grid, w.tile_shapes, w.scale)
+    Tg = T.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(Tg, T_o, rtol=2e-3, atol=1e-12)
+    np.testing.assert_allclose(lse.cpu().numpy(), lse_o, rtol=0, atol=ph.LSE_ABS)
+    # oracle mask = Top-k of the teacher rows, bit-exact where the gap is clear
+    prob = vb.Problem.from_workload(w)
+    mask = torch.empty((w.B, w.H, w.nT, w.nT), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((w.B, w.H, w.nT, w.k), dtype=torch.int32, device="cuda")
+    vb.veda_topk_mask(prob, T, mask, idx)
+    m_o, i_o = oracle.topk(T_o, w.k)
+    ph.check_masks(mask.cpu().numpy(), idx.cpu().numpy(), T_o, m_o, i_o, w.k)
+
+
+def test_recall_exact_on_given_lists(vb, oracle):
+    rng = np.random.default_rng(9)
+    w = workloads.custom("recall", 2, 3, 64, (1, 1, 64 * 50), [(1, 1, 64)], 9)
+    shape = (w.B, w.H, w.nT, w.k)
+    a = np.sort(np.stack([rng.permutation(w.nT)[:w.k] for _ in range(np.prod(shape[:-1]))]), 1)
+    b = np.sort(np.stack([rng.permutation(w.nT)[:w.k] for _ in range(np.prod(shape[:-1]))]), 1)
+    a, b = a.reshape(shape).astype(np.int32), b.reshape(shape).astype(np.int32)
+    b[0, 0, 0] = a[0, 0, 0]  # one row of full overlap
+    prob = vb.Problem.from_workload(w)
+    rows = torch.empty(shape[:-1], dtype=torch.float32, device="cuda")
+    mean = torch.empty((1,), dtype=torch.float64, device="cuda")
+    ws = vb.alloc_workspace(prob)
+    vb.veda_tile_recall(prob, torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda(), rows, mean, ws)
+    per_o, mean_o = oracle.tile_recall(a, b)
+    np.testing.assert_array_equal(rows.cpu().numpy(), per_o.astype(np.float32))
+    assert mean.item() == mean_o
+
+
+def test_recall_of_predicted_mask_against_oracle_mask(vb, oracle):
+    """End to end: Veda's predicted mask vs the teacher's oracle mask."""
+    w = workloads.custom("e2e", 1, 2, 128, (4, 16, 32), [(2, 8, 8)], 3)
+    t = {n: v.cuda() for n, v in workloads.generate(w, device="cpu").items()}
+    prob = vb.Problem.from_workload(w)
+    T, _, _ = _run_teacher(vb, w, t)
+    idx_oracle = torch.empty((w.B, w.H, w.nT, w.k), dtype=torch.int32, device="cuda")
+    vb.veda_topk_mask(prob, T, None, idx_oracle)
+    O = torch.empty_like(t["Q"])
+    idx_pred = torch.empty_like(idx_oracle)
+    ws = vb.alloc_workspace(prob)
+    vb.veda_forward(prob, t["Q"], t["K"], t["V"], t["Wq"], t["Wk"], O, None, idx_pred, None, ws)
+    mean = torch.empty((1,), dtype=torch.float64, device="cuda")
+    vb.veda_tile_recall(prob, idx_pred, idx_oracle, None, mean, ws)
+    Qb, Kb = ph.to_host_bits(t["Q"]), ph.to_host_bits(t["K"])
+    ora = oracle.mask_prep(Qb, Kb, t["Wq"].cpu().numpy(), t["Wk"].cpu().numpy(), w.grid,
+                           w.tile_shapes, w.k)
+    T_o, _ = oracle.teacher(Qb, Kb, w.grid, w.tile_shapes, w.scale)
+    _, i_o = oracle.topk(T_o, w.k)
+    _, mean_o = oracle.tile_recall(ora["idx"], i_o)
+    # rows whose selection is a near-tie may differ; each such row moves recall by <= 1/nrows
+    ex = ph.exempt_rows(ora["S"], w.k).sum() + ph.exempt_rows(T_o, w.k).sum()
+    assert abs(mean.item() - mean_o) <= ex / (w.B * w.H * w.nT) + 1e-12
+    assert 0.0 <= mean.item() <= 1.0

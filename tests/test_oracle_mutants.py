@@ -36,6 +36,7 @@ MUTANTS = {
     "max and min swapped": ("out[1 * d + c] = mx;\n            out[2 * d + c] = mn;",
                             "out[1 * d + c] = mn;\n            out[2 * d + c] = mx;"),
     "teacher average-pools": ("if (p > trow[j]) trow[j] = p;", "trow[j] += p / (double)Bt;"),
+    "recall counts predicted tiles twice": ("hits += found;", "hits += found + (a == 0);"),
 }
 
 
@@ -58,6 +59,8 @@ def pin_suite(o):
     yield lambda: pins.test_attention_1d_tiles_is_block_sparse(o)
     yield lambda: pins.test_attention_renormalisation(o)
     yield lambda: pins.test_teacher_is_tile_max_of_dense_probs(o, *pins.SMALL_CASES[0])
+    yield lambda: pins.test_tile_recall_hand_cases(o)
+    yield lambda: pins.test_tile_recall_brute_force(o)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -315,3 +315,25 @@ def test_generator_is_seeded():
         assert torch.equal(a[n], b[n])
     c = workloads.generate(workloads.tiny(seed=1))
     assert not torch.equal(a["Q"], c["Q"])
+
+
+# ---------------------------------------------------------------- tile recall
+def test_tile_recall_hand_cases(oracle):
+    pred = np.array([[0, 2, 5], [1, 2, 3], [4, 6, 7]], np.int32)
+    ref = np.array([[2, 3, 5], [1, 2, 3], [0, 1, 2]], np.int32)
+    per, mean = oracle.tile_recall(pred, ref)
+    np.testing.assert_array_equal(per, [2 / 3, 1.0, 0.0])
+    assert mean == (2 + 3 + 0) / 9
+
+
+def test_tile_recall_brute_force(oracle):
+    rng = np.random.default_rng(4)
+    nT, k = 40, 7
+    pred = np.sort(np.stack([rng.permutation(nT)[:k] for _ in range(50)]), 1).astype(np.int32)
+    ref = np.sort(np.stack([rng.permutation(nT)[:k] for _ in range(50)]), 1).astype(np.int32)
+    per, mean = oracle.tile_recall(pred, ref)
+    want = np.array([len(set(a) & set(b)) / k for a, b in zip(pred, ref)])
+    np.testing.assert_array_equal(per, want)
+    assert abs(mean - want.mean()) < 1e-15
+    per_self, mean_self = oracle.tile_recall(ref, ref)
+    assert mean_self == 1.0 and np.all(per_self == 1.0)

@@ -71,6 +71,10 @@ def load_library(path: str = LIB_PATH):
     lib.veda_forward.restype = st
     lib.veda_get_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32)]
     lib.veda_get_status.restype = st
+    lib.veda_teacher.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 8
+    lib.veda_teacher.restype = st
+    lib.veda_tile_recall.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 6
+    lib.veda_tile_recall.restype = st
     lib.veda_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.veda_tile_score_noalloc.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 6
     lib.veda_tile_score_noalloc.restype = st
@@ -182,6 +186,27 @@ def veda_forward(problem: Problem, Q, K, V, Wq, Wk, O, lse, idx_out, mask_out, w
     _check(load_library().veda_forward(ctypes.byref(problem.c), _ptr(Q), _ptr(K), _ptr(V),
                                        _ptr(Wq), _ptr(Wk), _ptr(O), _ptr(lse), _ptr(idx_out),
                                        _ptr(mask_out), _ptr(ws), _stream(stream)))
+
+
+def veda_teacher(problem: Problem, Q, K, V, O_dense, lse_dense, teacher, ws, stream=None) -> None:
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O_dense, "O_dense")):
+        _expect(t, torch.bfloat16, n)
+    for t, n in ((lse_dense, "lse_dense"), (teacher, "teacher")):
+        _expect(t, torch.float32, n)
+    _check(load_library().veda_teacher(ctypes.byref(problem.c), _ptr(Q), _ptr(K), _ptr(V),
+                                       _ptr(O_dense), _ptr(lse_dense), _ptr(teacher), _ptr(ws),
+                                       _stream(stream)))
+
+
+def veda_tile_recall(problem: Problem, idx_pred, idx_ref, recall_rows, recall_mean, ws,
+                     stream=None) -> None:
+    _expect(idx_pred, torch.int32, "idx_pred")
+    _expect(idx_ref, torch.int32, "idx_ref")
+    _expect(recall_rows, torch.float32, "recall_rows")
+    _expect(recall_mean, torch.float64, "recall_mean")
+    _check(load_library().veda_tile_recall(ctypes.byref(problem.c), _ptr(idx_pred), _ptr(idx_ref),
+                                           _ptr(recall_rows), _ptr(recall_mean), _ptr(ws),
+                                           _stream(stream)))
 
 
 def veda_get_status(ws, stream=None) -> int:

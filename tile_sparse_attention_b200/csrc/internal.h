@@ -55,6 +55,23 @@ veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint1
                                const uint16_t* V, const int32_t* idx, int k, uint16_t* O,
                                float* lse, int* status, cudaStream_t s);
 
+// TMA descriptors (tensor_maps.cu): the 5-D tile view (d, Ws, Hs, T, B*H) of a
+// [B,H,N,d] bf16 tensor with a (64, p_w, p_h, p_t, 1) box, and a 2-D row view
+// of an fp32 [rows][cols] matrix with a (32, 128) box; both 128-byte swizzled.
+veda_status encode_tile_map(CUtensorMap* map, const void* base, const Problem& pr,
+                            const int* shape);
+veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows, int cols);
+// Time limit of a device wait (VEDA_WAIT_LIMIT_MS, default 10 s).
+unsigned long long wait_limit_ns();
+
+// Max-pooled teacher (teacher.cu): T [B,H,nT,nT] from Q, K and the dense lse.
+veda_status launch_teacher(const Problem& pr, const uint16_t* Q, const uint16_t* K,
+                           const float* lse, float* teacher, int* status, cudaStream_t s);
+// Tile recall of idx_pred against idx_ref (both [B,H,nT,k], ascending rows);
+// scratch8: 8 bytes of device scratch for the hit counter.
+veda_status launch_recall(const Problem& pr, const int32_t* idx_pred, const int32_t* idx_ref,
+                          float* per_row, double* mean, void* scratch8, cudaStream_t s);
+
 // Workspace layout of veda_forward (byte offsets, 256-aligned).
 struct WorkspaceLayout {
     size_t status, statsQ, statsK, qt, kt, S, idx, total;

@@ -1,0 +1,66 @@
+// kernel_common.cuh -- device helpers shared by the tcgen05 kernels: bounded
+// mbarrier waits and tile geometry.
+#pragma once
+
+#include "../../include/veda.h"
+#include "ptx.cuh"
+
+namespace veda {
+
+// Suspend-time hint of one barrier test: the waiting warp sleeps in hardware
+// (woken as soon as the phase completes) instead of spinning.
+constexpr uint32_t kSuspendNs = 20000;
+
+// Bounded wait: false when the time limit expired (VEDA_ERR_TIMEOUT is then
+// recorded and the CTA's abort flag raised) or another role aborted.  P is a
+// kernel parameter struct with `status` and `wait_limit_ns` fields.
+template <class P>
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const P& p,
+                                         volatile int* abort_flag) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > p.wait_limit_ns) {
+            *abort_flag = 1;
+            atomicCAS(p.status, 0, (int)VEDA_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag (drain on the way out).
+template <class P>
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity, const P& p) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait_sleep(bar, parity, kSuspendNs)) {
+        if (global_timer_ns() - t0 > p.wait_limit_ns) {
+            atomicCAS(p.status, 0, (int)VEDA_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast and the
+// warp re-converges (the thread sync orders the other lanes after the wait).
+template <class P>
+__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity, const P& p,
+                                              volatile int* abort_flag) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, p, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// Grid origin (t0, y0, x0) of tile t for tile shape (pt, ph, pw).
+__device__ __forceinline__ void tile_origin(int t, int pt, int ph, int pw, int Hs, int Ws,
+                                            int& t0, int& y0, int& x0) {
+    const int nh = Hs / ph, nw = Ws / pw;
+    t0 = (t / (nh * nw)) * pt;
+    y0 = ((t / nw) % nh) * ph;
+    x0 = (t % nw) * pw;
+}
+
+}  // namespace veda

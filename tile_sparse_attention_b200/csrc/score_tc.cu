@@ -196,34 +196,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows, int kext) {
-    static EncodeTiledFn fn = nullptr;
-    if (fn == nullptr) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    if (fn == nullptr) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    const cuuint64_t dims[2] = {(cuuint64_t)kext, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)kext * 4};
-    const cuuint32_t box[2] = {32, 128};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
-        return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled (score) failed: " + std::to_string((int)r));
-    return VEDA_OK;
-}
-
 }  // namespace
 
 veda_status launch_score(const Problem& pr, const float* qext, const float* kext, float* S,
@@ -239,10 +211,7 @@ veda_status launch_score(const Problem& pr, const float* qext, const float* kext
     prm.status = status;
     prm.nT = pr.nT;
     prm.kblocks = kx / 32;
-    const char* env = getenv("VEDA_WAIT_LIMIT_MS");
-    unsigned long long ms = 10000ull;
-    if (env != nullptr && atoll(env) > 0) ms = (unsigned long long)atoll(env);
-    prm.wait_limit_ns = ms * 1000000ull;
+    prm.wait_limit_ns = wait_limit_ns();
     cudaError_t err = cudaFuncSetAttribute(score_tc_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return cuda_check(err, "score smem attribute");

@@ -39,6 +39,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "kernel_common.cuh"
 #include "ptx.cuh"
 
 namespace veda {
@@ -106,52 +107,6 @@ struct Bars {
     uint64_t* p_full;
     uint64_t* drain;
 };
-
-// Bounded wait: false when the limit expired or another role aborted.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const AttnParams& p,
-                                         volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > p.wait_limit_ns) {
-            *abort_flag = 1;
-            atomicCAS(p.status, 0, (int)VEDA_ERR_TIMEOUT);
-            return false;
-        }
-    }
-}
-
-// Bounded wait that ignores the abort flag (drain on the way out).
-__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity, const AttnParams& p) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > p.wait_limit_ns) {
-            atomicCAS(p.status, 0, (int)VEDA_ERR_TIMEOUT);
-            return;
-        }
-    }
-}
-
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast and the
-// warp re-converges (the thread sync orders the other lanes after the wait).
-__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
-                                              const AttnParams& p, volatile int* abort_flag) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, p, abort_flag) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    __syncwarp();
-    return ok != 0;
-}
-
-__device__ __forceinline__ void tile_origin(int t, int pt, int ph, int pw, int Hs, int Ws,
-                                            int& t0, int& y0, int& x0) {
-    const int nh = Hs / ph, nw = Ws / pw;
-    t0 = (t / (nh * nw)) * pt;
-    y0 = ((t / nw) % nh) * ph;
-    x0 = (t % nw) * pw;
-}
 
 // Barrier phase bookkeeping (each barrier completes once per use; b = j & 1,
 // m = j >> 1; stage st = j % NS holds K_j and V_j, fill n = j / NS):
@@ -541,46 +496,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (fn == nullptr) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// 5-D view (d, Ws, Hs, T, B*H) of a [B,H,N,d] bf16 tensor; box (64, pw, ph, pt, 1).
-veda_status encode_tile_map(CUtensorMap* map, const void* base, const Problem& pr,
-                            const int* shape) {
-    EncodeTiledFn enc = get_encode_fn();
-    if (enc == nullptr) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    const cuuint64_t dims[5] = {(cuuint64_t)pr.d, (cuuint64_t)pr.Ws, (cuuint64_t)pr.Hs,
-                                (cuuint64_t)pr.T, (cuuint64_t)pr.B * pr.H};
-    const cuuint64_t strides[4] = {(cuuint64_t)pr.d * 2, (cuuint64_t)pr.Ws * pr.d * 2,
-                                   (cuuint64_t)pr.Hs * pr.Ws * pr.d * 2,
-                                   (cuuint64_t)pr.N * pr.d * 2};
-    const cuuint32_t box[5] = {64, (cuuint32_t)shape[2], (cuuint32_t)shape[1],
-                               (cuuint32_t)shape[0], 1};
-    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
-        return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string((int)r));
-    return VEDA_OK;
-}
-
 template <int D, int BT, int NS>
 veda_status launch_cfg(const AttnParams& prm, const Problem& pr, cudaStream_t s) {
     using C = Cfg<D, BT, NS>;
@@ -592,13 +507,6 @@ veda_status launch_cfg(const AttnParams& prm, const Problem& pr, cudaStream_t s)
     dim3 grid(pr.nT, pr.B * pr.H);
     sparse_attn_kernel<D, BT, NS><<<grid, kThreads, C::kSmemBytes, s>>>(prm);
     return cuda_check(cudaGetLastError(), "sparse_attn launch");
-}
-
-unsigned long long wait_limit_ns() {
-    const char* env = getenv("VEDA_WAIT_LIMIT_MS");
-    unsigned long long ms = 10000ull;  // a healthy wait takes microseconds
-    if (env != nullptr && atoll(env) > 0) ms = (unsigned long long)atoll(env);
-    return ms * 1000000ull;
 }
 
 }  // namespace

@@ -234,6 +234,40 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
     return launch_sparse_attn(pr, Q, K, V, idx, pr.k, O, lse, status, s);
 }
 
+veda_status veda_teacher(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
+                         const uint16_t* V, uint16_t* O_dense, float* lse_dense, float* teacher,
+                         void* ws, veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, false, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(Q, "Q")) || (st = check_ptr(K, "K")) || (st = check_ptr(V, "V")) ||
+        (st = check_ptr(O_dense, "O_dense")) || (st = check_ptr(lse_dense, "lse_dense")) ||
+        (st = check_ptr(teacher, "teacher")) || (st = check_ptr(ws, "ws")))
+        return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    int* status = static_cast<int*>(ws);
+    if ((st = cuda_check(cudaMemsetAsync(status, 0, sizeof(int), s), "status reset"))) return st;
+    // dense schedule: every key tile, for the softmax normaliser of every row
+    if ((st = launch_sparse_attn(pr, Q, K, V, nullptr, pr.nT, O_dense, lse_dense, status, s)))
+        return st;
+    return launch_teacher(pr, Q, K, lse_dense, teacher, status, s);
+}
+
+veda_status veda_tile_recall(const veda_problem* p, const int32_t* idx_pred,
+                             const int32_t* idx_ref, float* recall_rows, double* recall_mean,
+                             void* ws, veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, true, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(idx_pred, "idx_pred")) || (st = check_ptr(idx_ref, "idx_ref")) ||
+        (st = check_ptr(recall_rows, "recall_rows", true)) ||
+        (st = check_ptr(recall_mean, "recall_mean")) || (st = check_ptr(ws, "ws")))
+        return st;
+    // the hit counter lives in the status area of the workspace, past the status word
+    return launch_recall(pr, idx_pred, idx_ref, recall_rows, recall_mean,
+                         static_cast<char*>(ws) + 128, (cudaStream_t)stream);
+}
+
 veda_status veda_get_status(const void* ws, veda_stream_t stream, int32_t* device_status) {
     if (ws == nullptr || device_status == nullptr)
         return fail(VEDA_ERR_INVALID_ARG, "ws and device_status must be non-NULL");
