@@ -187,6 +187,29 @@ veda_status veda_tile_recall(const veda_problem* p, const int32_t* idx_pred,
                              void* ws, veda_stream_t stream);
 
 /*
+ * KL structure distillation of the estimator (project page, "Principle 01
+ * Full-Attention Structure Distillation"; "Theoretical Rationale" 4,
+ * Distillation Objective: row-wise KL between the max-pooled teacher's tile
+ * distribution and the estimator's soft distribution over key tiles, before
+ * Top-k).  With R = B*H*nT rows:
+ *   A_tgt[i,:]  = teacher[i,:] / sum_j teacher[i,j]
+ *   A_pred[i,:] = softmax(S[i,:] / tau)
+ *   loss        = (1/R) sum_i KL(A_tgt[i] || A_pred[i])            (fp64, device)
+ *   dWq, dWk    = d loss / d Wq, d loss / d Wk  (fp32 [H, d, d]) through
+ *                 S = sum_s (statsQ_s Wq) . (statsK_s Wk)
+ *   S must be the score of (statsQ, statsK, Wq, Wk) (veda_tile_score);
+ *   teacher: fp32 [B, H, nT, nT], rows with a positive sum (veda_teacher).
+ *   tau > 0; nT must be a multiple of 8.
+ *   ws: at least veda_distill_workspace_size() bytes.
+ * fp32 arithmetic with fp64 row sums; the loss is reduced in a fixed order.
+ */
+veda_status veda_distill_workspace_size(const veda_problem* p, size_t* bytes);
+veda_status veda_distill_kl(const veda_problem* p, const float* statsQ, const float* statsK,
+                            const float* Wq, const float* Wk, const float* S, const float* teacher,
+                            float tau, double* loss, float* dWq, float* dWk, void* ws,
+                            veda_stream_t stream);
+
+/*
  * Waits for `stream`, then copies the device status word of `ws` into
  * *device_status (VEDA_OK or a device-detected veda_status code).
  */

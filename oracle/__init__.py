@@ -58,6 +58,8 @@ def _bind(lib):
     lib.oracle_teacher.argtypes = [_I64] * 6 + [_P, ctypes.c_double, _P, _P, _P, _P]
     lib.oracle_tile_recall.argtypes = [_I64, _I64, _P, _P, _P]
     lib.oracle_tile_recall.restype = ctypes.c_double
+    lib.oracle_distill_kl.argtypes = [_I64] * 4 + [_P] * 5 + [ctypes.c_double, _P, _P]
+    lib.oracle_distill_kl.restype = ctypes.c_double
     return lib
 
 
@@ -207,3 +209,19 @@ class Oracle:
         per = np.empty(a.shape[:-1], dtype=np.float64)
         mean = self.lib.oracle_tile_recall(rows, k, _ptr(a), _ptr(b), _ptr(per))
         return per, float(mean)
+
+    def distill_kl(self, statsQ, statsK, Wq, Wk, teacher, tau, grads=True):
+        """KL distillation loss (mean over rows) and, optionally, dL/dWq, dL/dWk."""
+        sq = np.ascontiguousarray(statsQ, dtype=np.float64)
+        sk = np.ascontiguousarray(statsK, dtype=np.float64)
+        Wq = np.ascontiguousarray(Wq, dtype=np.float32)
+        Wk = np.ascontiguousarray(Wk, dtype=np.float32)
+        T = np.ascontiguousarray(teacher, dtype=np.float64)
+        B, H, nT, _, d = sq.shape
+        dWq = np.empty((H, d, d), dtype=np.float64) if grads else None
+        dWk = np.empty((H, d, d), dtype=np.float64) if grads else None
+        loss = self.lib.oracle_distill_kl(B, H, nT, d, _ptr(sq), _ptr(sk), _ptr(Wq), _ptr(Wk),
+                                          _ptr(T), float(tau),
+                                          _ptr(dWq) if grads else None,
+                                          _ptr(dWk) if grads else None)
+        return (float(loss), dWq, dWk) if grads else float(loss)

@@ -384,3 +384,96 @@ double oracle_tile_recall(int64_t rows, int64_t k, const int32_t* pred, const in
     }
     return total / ((double)rows * (double)k);
 }
+
+/*
+ * KL structure distillation (Principle 01, "Full-Attention Structure
+ * Distillation"; Theoretical Rationale 4, "Distillation Objective": row-wise
+ * KL between the teacher's tile distribution and the estimator's soft
+ * distribution over key tiles).  Readings: the target row is the teacher row
+ * divided by its sum; the prediction is softmax(S / tau); the loss is the mean
+ * of the row divergences over all B*H*nT rows.
+ *   statsQ, statsK: [B, H, nT, 3, d];  Wq, Wk: [H, d, d] fp32
+ *   teacher: [B, H, nT, nT];  dWq, dWk: [H, d, d] (may be NULL)
+ * Returns the loss.  The gradient follows the chain rule through
+ * S = sum_s (statsQ_s Wq) . (statsK_s Wk):
+ *   dS = (pred - tgt) / (tau R);  dq~ = dS k~;  dk~ = dS^T q~;
+ *   dWq = sum stats_Q^T dq~;  dWk = sum stats_K^T dk~.
+ */
+double oracle_distill_kl(int64_t B, int64_t H, int64_t nT, int64_t d,
+                         const double* statsQ, const double* statsK, const float* Wq,
+                         const float* Wk, const double* teacher, double tau,
+                         double* dWq, double* dWk) {
+    int64_t n3 = B * H * nT * 3 * d;
+    double* qt = (double*)malloc(sizeof(double) * (size_t)n3);
+    double* kt = (double*)malloc(sizeof(double) * (size_t)n3);
+    double* S = (double*)malloc(sizeof(double) * (size_t)(B * H * nT * nT));
+    double* G = (double*)malloc(sizeof(double) * (size_t)(B * H * nT * nT));
+    oracle_project(B, H, nT, d, statsQ, Wq, qt);
+    oracle_project(B, H, nT, d, statsK, Wk, kt);
+    oracle_score(B, H, nT, d, qt, kt, S);
+    int64_t R = B * H * nT;
+    double total = 0.0;
+    for (int64_t row = 0; row < R; ++row) {
+        const double* s = S + row * nT;
+        const double* t = teacher + row * nT;
+        double mx = -INFINITY, tsum = 0.0;
+        for (int64_t j = 0; j < nT; ++j) {
+            if (s[j] / tau > mx) mx = s[j] / tau;
+            tsum += t[j];
+        }
+        double se = 0.0;
+        for (int64_t j = 0; j < nT; ++j) se += exp(s[j] / tau - mx);
+        double lse = mx + log(se);
+        double kl = 0.0;
+        for (int64_t j = 0; j < nT; ++j) {
+            double logp = s[j] / tau - lse;
+            double tg = t[j] / tsum;
+            if (tg > 0.0) kl += tg * (log(tg) - logp);
+            G[row * nT + j] = (exp(logp) - tg) / (tau * (double)R);
+        }
+        total += kl;
+    }
+    if (dWq && dWk) {
+        for (int64_t e = 0; e < H * d * d; ++e) {
+            dWq[e] = 0.0;
+            dWk[e] = 0.0;
+        }
+        double* dq = (double*)malloc(sizeof(double) * (size_t)(3 * d));
+        double* dk = (double*)malloc(sizeof(double) * (size_t)(3 * d));
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t h = 0; h < H; ++h) {
+                int64_t bh = b * H + h;
+                for (int64_t i = 0; i < nT; ++i) {
+                    /* dq~_i = sum_j G[i,j] k~_j ;  dk~_i = sum_j G[j,i] q~_j */
+                    for (int64_t c = 0; c < 3 * d; ++c) {
+                        dq[c] = 0.0;
+                        dk[c] = 0.0;
+                    }
+                    for (int64_t j = 0; j < nT; ++j) {
+                        double gij = G[(bh * nT + i) * nT + j];
+                        double gji = G[(bh * nT + j) * nT + i];
+                        for (int64_t c = 0; c < 3 * d; ++c) {
+                            dq[c] += gij * kt[(bh * nT + j) * 3 * d + c];
+                            dk[c] += gji * qt[(bh * nT + j) * 3 * d + c];
+                        }
+                    }
+                    for (int64_t s3 = 0; s3 < 3; ++s3) {
+                        const double* sq = statsQ + ((bh * nT + i) * 3 + s3) * d;
+                        const double* sk = statsK + ((bh * nT + i) * 3 + s3) * d;
+                        for (int64_t ci = 0; ci < d; ++ci)
+                            for (int64_t co = 0; co < d; ++co) {
+                                dWq[(h * d + ci) * d + co] += sq[ci] * dq[s3 * d + co];
+                                dWk[(h * d + ci) * d + co] += sk[ci] * dk[s3 * d + co];
+                            }
+                    }
+                }
+            }
+        free(dq);
+        free(dk);
+    }
+    free(qt);
+    free(kt);
+    free(S);
+    free(G);
+    return total / (double)R;
+}

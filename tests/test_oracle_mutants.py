@@ -37,6 +37,16 @@ MUTANTS = {
                             "out[1 * d + c] = mn;\n            out[2 * d + c] = mx;"),
     "teacher average-pools": ("if (p > trow[j]) trow[j] = p;", "trow[j] += p / (double)Bt;"),
     "recall counts predicted tiles twice": ("hits += found;", "hits += found + (a == 0);"),
+    "distillation gradient has the wrong sign": (
+        "G[row * nT + j] = (exp(logp) - tg) / (tau * (double)R);",
+        "G[row * nT + j] = (tg - exp(logp)) / (tau * (double)R);"),
+    "distillation gradient drops the temperature": (
+        "G[row * nT + j] = (exp(logp) - tg) / (tau * (double)R);",
+        "G[row * nT + j] = (exp(logp) - tg) / ((double)R);"),
+    "distillation uses the key stats for dWq": (
+        "dWq[(h * d + ci) * d + co] += sq[ci] * dq[s3 * d + co];",
+        "dWq[(h * d + ci) * d + co] += sk[ci] * dq[s3 * d + co];"),
+    "distillation target not normalised": ("double tg = t[j] / tsum;", "double tg = t[j];"),
 }
 
 
@@ -61,6 +71,9 @@ def pin_suite(o):
     yield lambda: pins.test_teacher_is_tile_max_of_dense_probs(o, *pins.SMALL_CASES[0])
     yield lambda: pins.test_tile_recall_hand_cases(o)
     yield lambda: pins.test_tile_recall_brute_force(o)
+    yield lambda: pins.test_distill_gradient_matches_finite_differences(o, 0.7, 1)
+    yield lambda: pins.test_distill_zero_when_target_equals_prediction(o)
+    yield lambda: pins.test_distill_invariances_and_positivity(o)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -337,3 +337,58 @@ def test_tile_recall_brute_force(oracle):
     assert abs(mean - want.mean()) < 1e-15
     per_self, mean_self = oracle.tile_recall(ref, ref)
     assert mean_self == 1.0 and np.all(per_self == 1.0)
+
+
+# ---------------------------------------------------------------- KL distillation
+def _distill_case(seed=0, B=1, H=2, nT=6, d=4):
+    rng = np.random.default_rng(seed)
+    sq = rng.standard_normal((B, H, nT, 3, d))
+    sk = rng.standard_normal((B, H, nT, 3, d))
+    Wq = (rng.standard_normal((H, d, d)) / 2).astype(np.float32)
+    Wk = (rng.standard_normal((H, d, d)) / 2).astype(np.float32)
+    T = rng.uniform(0.01, 1.0, (B, H, nT, nT))
+    return sq, sk, Wq, Wk, T
+
+
+@pytest.mark.parametrize("tau,B", [(0.7, 1), (1.0, 2), (3.0, 1)])
+def test_distill_gradient_matches_finite_differences(oracle, tau, B):
+    """Central differences of the loss (computed from its definition) pin dL/dW."""
+    sq, sk, Wq, Wk, T = _distill_case(B=B)
+    _, dWq, dWk = oracle.distill_kl(sq, sk, Wq, Wk, T, tau)
+    scale = max(np.abs(dWq).max(), np.abs(dWk).max())
+    eps = np.float32(2.0 ** -12)
+    for side in ("q", "k"):
+        W, dW = (Wq, dWq) if side == "q" else (Wk, dWk)
+        for (h, a, b) in [(0, 0, 0), (1, 2, 3), (0, 3, 1), (1, 1, 2), (0, 2, 2)]:
+            Wp, Wm = W.copy(), W.copy()
+            Wp[h, a, b] = np.float32(W[h, a, b] + eps)
+            Wm[h, a, b] = np.float32(W[h, a, b] - eps)
+            step = float(Wp[h, a, b]) - float(Wm[h, a, b])
+            args_p = (Wp, Wk) if side == "q" else (Wq, Wp)
+            args_m = (Wm, Wk) if side == "q" else (Wq, Wm)
+            Lp = oracle.distill_kl(sq, sk, *args_p, T, tau, grads=False)
+            Lm = oracle.distill_kl(sq, sk, *args_m, T, tau, grads=False)
+            fd = (Lp - Lm) / step
+            assert abs(fd - dW[h, a, b]) <= 1e-4 * scale + 1e-10, (side, h, a, b, fd, dW[h, a, b])
+
+
+def test_distill_zero_when_target_equals_prediction(oracle):
+    sq, sk, Wq, Wk, _ = _distill_case(seed=3)
+    tau = 1.7
+    S = oracle.score(oracle.project(sq, Wq), oracle.project(sk, Wk))
+    T = np.exp(S / tau - (S / tau).max(-1, keepdims=True)) * 5.0  # any positive row scale
+    L, dWq, dWk = oracle.distill_kl(sq, sk, Wq, Wk, T, tau)
+    assert abs(L) < 1e-14
+    assert np.abs(dWq).max() < 1e-12 and np.abs(dWk).max() < 1e-12
+
+
+def test_distill_invariances_and_positivity(oracle):
+    sq, sk, Wq, Wk, T = _distill_case(seed=5)
+    L = oracle.distill_kl(sq, sk, Wq, Wk, T, 1.0, grads=False)
+    assert L > 0
+    # the teacher enters only through its row-normalised distribution
+    T2 = T * np.random.default_rng(1).uniform(0.5, 3.0, T.shape[:-1] + (1,))
+    assert abs(oracle.distill_kl(sq, sk, Wq, Wk, T2, 1.0, grads=False) - L) < 1e-13
+    # S / tau is what matters: scaling Wq by 2 and tau by 2 leaves the loss unchanged
+    L2 = oracle.distill_kl(sq, sk, (Wq * 2).astype(np.float32), Wk, T, 2.0, grads=False)
+    assert abs(L2 - L) < 1e-12

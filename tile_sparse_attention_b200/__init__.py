@@ -75,6 +75,12 @@ def load_library(path: str = LIB_PATH):
     lib.veda_teacher.restype = st
     lib.veda_tile_recall.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 6
     lib.veda_tile_recall.restype = st
+    lib.veda_distill_workspace_size.argtypes = [ctypes.POINTER(veda_problem),
+                                                ctypes.POINTER(ctypes.c_size_t)]
+    lib.veda_distill_workspace_size.restype = st
+    lib.veda_distill_kl.argtypes = ([ctypes.POINTER(veda_problem)] + [_P] * 6 + [ctypes.c_float]
+                                    + [_P] * 4 + [_P])
+    lib.veda_distill_kl.restype = st
     lib.veda_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.veda_tile_score_noalloc.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 6
     lib.veda_tile_score_noalloc.restype = st
@@ -207,6 +213,24 @@ def veda_tile_recall(problem: Problem, idx_pred, idx_ref, recall_rows, recall_me
     _check(load_library().veda_tile_recall(ctypes.byref(problem.c), _ptr(idx_pred), _ptr(idx_ref),
                                            _ptr(recall_rows), _ptr(recall_mean), _ptr(ws),
                                            _stream(stream)))
+
+
+def veda_distill_workspace_size(problem: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().veda_distill_workspace_size(ctypes.byref(problem.c), ctypes.byref(n)))
+    return int(n.value)
+
+
+def veda_distill_kl(problem: Problem, statsQ, statsK, Wq, Wk, S, teacher, tau, loss, dWq, dWk,
+                    ws, stream=None) -> None:
+    for t, n in ((statsQ, "statsQ"), (statsK, "statsK"), (Wq, "Wq"), (Wk, "Wk"), (S, "S"),
+                 (teacher, "teacher"), (dWq, "dWq"), (dWk, "dWk")):
+        _expect(t, torch.float32, n)
+    _expect(loss, torch.float64, "loss")
+    _check(load_library().veda_distill_kl(ctypes.byref(problem.c), _ptr(statsQ), _ptr(statsK),
+                                          _ptr(Wq), _ptr(Wk), _ptr(S), _ptr(teacher),
+                                          ctypes.c_float(tau), _ptr(loss), _ptr(dWq), _ptr(dWk),
+                                          _ptr(ws), _stream(stream)))
 
 
 def veda_get_status(ws, stream=None) -> int:

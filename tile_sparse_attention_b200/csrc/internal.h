@@ -64,6 +64,14 @@ veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows,
 // Time limit of a device wait (VEDA_WAIT_LIMIT_MS, default 10 s).
 unsigned long long wait_limit_ns();
 
+// Batched fp32 SIMT GEMM (tile_score.cu): C[z] (+)= op(A[z']) . op(B[z''])
+// with z' = z % a_batch_mod, z'' = z % b_batch_mod (when > 0); a_t: A stored
+// K x M; b_t: B stored N x K.  K must be a multiple of 8.
+veda_status launch_sgemm(const float* A, const float* B, float* C, int M, int N, int K, int lda,
+                         int ldb, int ldc, long long strideA, long long strideB, long long strideC,
+                         int batches, int a_batch_mod, int b_batch_mod, bool a_t, bool b_t,
+                         bool accumulate, cudaStream_t s);
+
 // Max-pooled teacher (teacher.cu): T [B,H,nT,nT] from Q, K and the dense lse.
 veda_status launch_teacher(const Problem& pr, const uint16_t* Q, const uint16_t* K,
                            const float* lse, float* teacher, int* status, cudaStream_t s);
@@ -71,6 +79,16 @@ veda_status launch_teacher(const Problem& pr, const uint16_t* Q, const uint16_t*
 // scratch8: 8 bytes of device scratch for the hit counter.
 veda_status launch_recall(const Problem& pr, const int32_t* idx_pred, const int32_t* idx_ref,
                           float* per_row, double* mean, void* scratch8, cudaStream_t s);
+
+// KL structure distillation (distill.cu).
+struct DistillLayout {
+    size_t qt, kt, dq, dk, G, row_kl, total;
+};
+DistillLayout distill_layout(const Problem& pr);
+veda_status launch_distill(const Problem& pr, const float* statsQ, const float* statsK,
+                           const float* Wq, const float* Wk, const float* S, const float* teacher,
+                           float tau, double* loss, float* dWq, float* dWk, void* ws,
+                           cudaStream_t s);
 
 // Workspace layout of veda_forward (byte offsets, 256-aligned).
 struct WorkspaceLayout {

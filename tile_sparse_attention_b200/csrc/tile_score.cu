@@ -33,6 +33,8 @@ struct GemmParams {
     int b_batch_mod;                      // >0: B index = batch % b_batch_mod
     int split;                            // 0: plain C; 1: query-side split; 2: key-side split
     int d;                                // head dimension (split layouts)
+    int accumulate;                       // plain C only: C += A . B
+    int a_batch_mod;                      // >0: A index = batch % a_batch_mod
 };
 
 // x = hi + lo with hi = x rounded to nearest TF32 (10 explicit mantissa bits)
@@ -43,13 +45,15 @@ __device__ __forceinline__ float tf32_hi(float x) {
 
 // C[z] = A[z] . B[z]  (B_T = false: B is K x N row-major)
 // C[z] = A[z] . B[z]^T (B_T = true: B is N x K row-major)
-template <bool B_T>
+// A_T = true: A is stored K x M row-major (C = A^T . B).  K is a multiple of 8.
+template <bool B_T, bool A_T = false>
 __global__ void __launch_bounds__(256) sgemm_kernel(const __grid_constant__ GemmParams p) {
     __shared__ __align__(16) float As[2][BK][BM + PAD];
     __shared__ __align__(16) float Bs[2][BK][BN + PAD];
 
     const int z = blockIdx.z;
-    const float* A = p.A + (long long)z * p.strideA;
+    const int az = p.a_batch_mod > 0 ? z % p.a_batch_mod : z;
+    const float* A = p.A + (long long)az * p.strideA;
     const int bz = p.b_batch_mod > 0 ? z % p.b_batch_mod : z;
     const float* Bm = p.B + (long long)bz * p.strideB;
     float* C = p.C + (long long)z * p.strideC;
@@ -63,9 +67,16 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const __grid_constant__ Gemm
     float4 ra, rb;
 
     auto load_a = [&](int k0) {
-        const int m = m0 + a_row;
-        ra = (m < p.M) ? *reinterpret_cast<const float4*>(A + (long long)m * p.lda + k0 + a_k)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (A_T) {
+            const int m = m0 + bn_n;
+            ra = (m < p.M)
+                     ? *reinterpret_cast<const float4*>(A + (long long)(k0 + bn_k) * p.lda + m)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            const int m = m0 + a_row;
+            ra = (m < p.M) ? *reinterpret_cast<const float4*>(A + (long long)m * p.lda + k0 + a_k)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     };
     auto load_b = [&](int k0) {
         if (B_T) {
@@ -80,10 +91,14 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const __grid_constant__ Gemm
         }
     };
     auto store_tiles = [&](int buf) {
-        As[buf][a_k + 0][a_row] = ra.x;
-        As[buf][a_k + 1][a_row] = ra.y;
-        As[buf][a_k + 2][a_row] = ra.z;
-        As[buf][a_k + 3][a_row] = ra.w;
+        if (A_T) {
+            *reinterpret_cast<float4*>(&As[buf][bn_k][bn_n]) = ra;
+        } else {
+            As[buf][a_k + 0][a_row] = ra.x;
+            As[buf][a_k + 1][a_row] = ra.y;
+            As[buf][a_k + 2][a_row] = ra.z;
+            As[buf][a_k + 3][a_row] = ra.w;
+        }
         if (B_T) {
             Bs[buf][a_k + 0][a_row] = rb.x;
             Bs[buf][a_k + 1][a_row] = rb.y;
@@ -155,10 +170,15 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const __grid_constant__ Gemm
             }
             float* dst = C + (long long)m * p.ldc + n;
             if (vec && n + 3 < p.N) {
-                *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+                float4 o = make_float4(v[0], v[1], v[2], v[3]);
+                if (p.accumulate) {
+                    const float4 c = *reinterpret_cast<const float4*>(dst);
+                    o.x += c.x; o.y += c.y; o.z += c.z; o.w += c.w;
+                }
+                *reinterpret_cast<float4*>(dst) = o;
             } else {
                 for (int e = 0; e < 4; ++e)
-                    if (n + e < p.N) dst[e] = v[e];
+                    if (n + e < p.N) dst[e] = p.accumulate ? dst[e] + v[e] : v[e];
             }
         }
     }
@@ -187,6 +207,36 @@ veda_status launch_project(const Problem& pr, const float* stats, const float* W
     dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM, pr.B * pr.H);
     sgemm_kernel<false><<<grid, 256, 0, s>>>(g);
     return cuda_check(cudaGetLastError(), "projection launch");
+}
+
+veda_status launch_sgemm(const float* A, const float* B, float* C, int M, int N, int K, int lda,
+                         int ldb, int ldc, long long strideA, long long strideB, long long strideC,
+                         int batches, int a_batch_mod, int b_batch_mod, bool a_t, bool b_t,
+                         bool accumulate, cudaStream_t s) {
+    if (K % 8 != 0 || lda % 4 != 0 || ldb % 4 != 0)
+        return fail(VEDA_ERR_UNSUPPORTED, "fp32 GEMM needs K and leading dimensions divisible by 8/4");
+    GemmParams g{};
+    g.A = A;
+    g.B = B;
+    g.C = C;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.lda = lda;
+    g.ldb = ldb;
+    g.ldc = ldc;
+    g.strideA = strideA;
+    g.strideB = strideB;
+    g.strideC = strideC;
+    g.a_batch_mod = a_batch_mod;
+    g.b_batch_mod = b_batch_mod;
+    g.accumulate = accumulate ? 1 : 0;
+    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, batches);
+    if (a_t && !b_t) sgemm_kernel<false, true><<<grid, 256, 0, s>>>(g);
+    else if (!a_t && b_t) sgemm_kernel<true, false><<<grid, 256, 0, s>>>(g);
+    else if (!a_t && !b_t) sgemm_kernel<false, false><<<grid, 256, 0, s>>>(g);
+    else return fail(VEDA_ERR_UNSUPPORTED, "fp32 GEMM: A and B both transposed");
+    return cuda_check(cudaGetLastError(), "fp32 GEMM launch");
 }
 
 }  // namespace veda

@@ -268,6 +268,34 @@ veda_status veda_tile_recall(const veda_problem* p, const int32_t* idx_pred,
                          static_cast<char*>(ws) + 128, (cudaStream_t)stream);
 }
 
+veda_status veda_distill_workspace_size(const veda_problem* p, size_t* bytes) {
+    Problem pr;
+    veda_status st = make_problem(p, false, &pr);
+    if (st != VEDA_OK) return st;
+    if (bytes == nullptr) return fail(VEDA_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = distill_layout(pr).total;
+    return VEDA_OK;
+}
+
+veda_status veda_distill_kl(const veda_problem* p, const float* statsQ, const float* statsK,
+                            const float* Wq, const float* Wk, const float* S, const float* teacher,
+                            float tau, double* loss, float* dWq, float* dWk, void* ws,
+                            veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, false, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(statsQ, "statsQ")) || (st = check_ptr(statsK, "statsK")) ||
+        (st = check_ptr(Wq, "Wq")) || (st = check_ptr(Wk, "Wk")) || (st = check_ptr(S, "S")) ||
+        (st = check_ptr(teacher, "teacher")) || (st = check_ptr(loss, "loss", false)) ||
+        (st = check_ptr(dWq, "dWq")) || (st = check_ptr(dWk, "dWk")) || (st = check_ptr(ws, "ws")))
+        return st;
+    if (!(tau > 0.f) || !isfinite(tau))
+        return fail(VEDA_ERR_INVALID_ARG, "tau must be positive and finite");
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((st = cuda_check(cudaMemsetAsync(ws, 0, sizeof(int), s), "status reset"))) return st;
+    return launch_distill(pr, statsQ, statsK, Wq, Wk, S, teacher, tau, loss, dWq, dWk, ws, s);
+}
+
 veda_status veda_get_status(const void* ws, veda_stream_t stream, int32_t* device_status) {
     if (ws == nullptr || device_status == nullptr)
         return fail(VEDA_ERR_INVALID_ARG, "ws and device_status must be non-NULL");
