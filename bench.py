@@ -360,7 +360,8 @@ def run_veda(args, w, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": dict(w.describe(), parallelism="replicas (one layer per GPU)" if world > 1
-                           else "single GPU", l2="inputs larger than L2 (Q/K/V 6.0 GB)"),
+                           else "single GPU",
+                           l2=f"inputs larger than L2 (Q/K/V {3 * B * H * N * d * 2 / 1e9:.2f} GB)"),
             "ms_per_layer": ms,
             "frac_of_peak": {"measured_bf16_burst": value / world / peaks["bf16"],
                              "measured_bf16_sustained": value / world / peaks["bf16_sus"],
@@ -386,6 +387,87 @@ def run_veda(args, w, world, rank, local):
     return 0
 
 
+# ---------------------------------------------------------------- next rows
+def run_rows(args, w, rows):
+    """Times the training-side rows on `w` (one JSON line per row)."""
+    import tile_sparse_attention_b200 as vb
+    vb.load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    t = workloads.generate(w, device=dev)
+    prob = vb.Problem.from_workload(w)
+    B, H, N, d, nT, k = w.B, w.H, w.N, w.d, w.nT, w.k
+    ws = vb.alloc_workspace(prob, dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = _peaks()
+
+    def timed(fn, reps=3):
+        fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps
+
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    T = torch.empty((B, H, nT, nT), dtype=torch.float32, device=dev)
+    dense_flops = w.dense_flops()
+    qk_flops = dense_flops / 2
+    if "f1" in rows:
+        ms_teacher = timed(lambda: vb.veda_teacher(prob, t["Q"], t["K"], t["V"], O, lse, T, ws))
+        ms_dense = timed(lambda: vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], None, O, lse, ws))
+        idx_o = torch.empty((B, H, nT, k), dtype=torch.int32, device=dev)
+        idx_p = torch.empty_like(idx_o)
+        ms_mask = timed(lambda: vb.veda_topk_mask(prob, T, None, idx_o))
+        vb.veda_forward(prob, t["Q"], t["K"], t["V"], t["Wq"], t["Wk"], O, None, idx_p, None, ws)
+        mean = torch.empty((1,), dtype=torch.float64, device=dev)
+        ms_rec = timed(lambda: vb.veda_tile_recall(prob, idx_p, idx_o, None, mean, ws))
+        ms_qk = ms_teacher - ms_dense
+        print(json.dumps({"row": "f1 teacher + oracle mask + tile recall", "workload": w.name,
+                          "teacher_ms": ms_teacher, "dense_attention_ms": ms_dense,
+                          "teacher_qk_pass_ms": ms_qk,
+                          "teacher_qk_TFLOP_s": qk_flops / (ms_qk * 1e-3) / 1e12,
+                          "frac_bf16_burst": qk_flops / (ms_qk * 1e-3) / 1e12 / peaks["bf16"],
+                          "oracle_mask_ms": ms_mask, "recall_ms": ms_rec,
+                          "tile_recall_random_weights": mean.item(),
+                          "status": vb.veda_get_status(ws)}), flush=True)
+    if "f3" in rows:
+        statsQ = torch.empty((B, H, nT, 3, d), dtype=torch.float32, device=dev)
+        statsK = torch.empty_like(statsQ)
+        S = torch.empty((B, H, nT, nT), dtype=torch.float32, device=dev)
+        vb.veda_tripool(prob, t["Q"], t["K"], statsQ, statsK)
+        vb.veda_tile_score(prob, statsQ, statsK, t["Wq"], t["Wk"], S, ws)
+        vb.veda_teacher(prob, t["Q"], t["K"], t["V"], O, lse, T, ws)
+        loss = torch.empty((1,), dtype=torch.float64, device=dev)
+        dWq, dWk = torch.empty_like(t["Wq"]), torch.empty_like(t["Wk"])
+        dws = torch.empty(vb.veda_distill_workspace_size(prob), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: vb.veda_distill_kl(prob, statsQ, statsK, t["Wq"], t["Wk"], S, T, 1.0,
+                                              loss, dWq, dWk, dws))
+        gflop = 2 * B * H * (2 * 3 * nT * d * d + 2 * nT * nT * 3 * d + 2 * 3 * nT * d * d) / 1e9
+        print(json.dumps({"row": "f3 KL distillation loss + dWq/dWk", "workload": w.name,
+                          "ms": ms, "fp32_GFLOP": gflop,
+                          "fp32_TFLOP_s": gflop / ms, "loss": loss.item(),
+                          "status": vb.veda_get_status(dws)}), flush=True)
+    if "f2" in rows:
+        cands = [c for c in workloads.HEAD_SHAPES
+                 if w.T % c[0] == 0 and w.Hs % c[1] == 0 and w.Ws % c[2] == 0]
+        Oc = torch.empty_like(t["Q"])
+        err = torch.empty((len(cands), B, H), dtype=torch.float64, device=dev)
+        best = torch.empty((H,), dtype=torch.int32, device=dev)
+        p0 = vb.Problem(B, H, d, w.grid, [cands[0]], k)
+        ms = timed(lambda: vb.veda_tile_search(p0, cands, t["Q"], t["K"], t["V"], t["Wq"],
+                                               t["Wk"], O, Oc, err, best, ws), reps=2)
+        picks = np.bincount(best.cpu().numpy(), minlength=len(cands)).tolist()
+        print(json.dumps({"row": "f2 head-aware tile search", "workload": w.name,
+                          "candidates": cands, "ms": ms, "heads_per_candidate": picks,
+                          "status": vb.veda_get_status(ws)}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -397,6 +479,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--rows", default="",
+                    help="comma list of f1,f2,f3: time the training-side rows instead")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "veda":
         args.warmup = 3
@@ -405,6 +489,8 @@ def main():
         w = workloads.sweep(int(T), int(s))
     else:
         w = workloads.CONFIGS[args.workload]()
+    if args.rows:
+        return run_rows(args, w, set(args.rows.split(",")))
     world, rank, local = _dist_init()
     try:
         if args.impl == "reference":

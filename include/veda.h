@@ -157,6 +157,26 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
                          veda_stream_t stream);
 
 /*
+ * Head-aware tile search (project page, "Head-Aware Tile Search"; "Principle
+ * 02 Head-Conditioned Tile Geometry"): for each head, the candidate tiling pi
+ * (p_t, p_h, p_w with the same product) that minimises
+ * ||O_full - O_sparse(pi)||_F^2 over the calibration batch.
+ *   p->tile_shapes is ignored; candidates: HOST int32 [ncand][3], 1 <= ncand <= 16,
+ *   each valid for the grid, all with the same p_t*p_h*p_w.
+ *   O_dense: bf16 [B, H, N, d], the full attention (dense schedule)
+ *   O_cand : bf16 [B, H, N, d] scratch (the layer output of the last candidate)
+ *   err    : fp64 [ncand, B, H], sum over tokens and channels of (O_dense - O_cand)^2
+ *   best   : int32 [H], argmin over candidates of the sum over B of err (ties: lower index)
+ *   ws     : at least veda_workspace_size() bytes (of `p` with any candidate)
+ * Each candidate runs the whole layer (veda_forward) on every head.
+ */
+veda_status veda_tile_search(const veda_problem* p, const int32_t* candidates, int32_t ncand,
+                             const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                             const float* Wq, const float* Wk, uint16_t* O_dense,
+                             uint16_t* O_cand, double* err, int32_t* best, void* ws,
+                             veda_stream_t stream);
+
+/*
  * Max-pooled full-attention teacher (project page, "Attention Structure
  * Distillation", Teacher; "Empirical Study" 02, Controlled Mask Intervention):
  *   teacher[b,h,i,j] = max over query tokens q of tile i and key tokens of

@@ -225,3 +225,45 @@ class Oracle:
                                           _ptr(dWq) if grads else None,
                                           _ptr(dWk) if grads else None)
         return (float(loss), dWq, dWk) if grads else float(loss)
+
+    def full_attention(self, Q, K, V, grid, tile_shapes, scale):
+        """Dense softmax attention for every token: O [B,H,N,d] fp64, lse [B,H,N]."""
+        Qb = _bf16_bits(Q)
+        B, H, N, d = Qb.shape
+        s = _shapes(tile_shapes)
+        nT = N // int(np.prod(s[0]))
+        idx = np.broadcast_to(np.arange(nT, dtype=np.int32), (B, H, nT, nT)).copy()
+        O, lse, toks = self.sparse_attention(Q, K, V, idx, grid, tile_shapes, scale)
+        return self._scatter(O, lse, toks, B, H, N, d, nT)
+
+    @staticmethod
+    def _scatter(O, lse, toks, B, H, N, d, nT):
+        Of = np.empty((B, H, N, d))
+        lf = np.empty((B, H, N))
+        u = 0
+        for b in range(B):
+            for h in range(H):
+                for i in range(nT):
+                    Of[b, h, toks[u]] = O[u]
+                    lf[b, h, toks[u]] = lse[u]
+                    u += 1
+        return Of, lf
+
+    def tile_search(self, Q, K, V, Wq, Wk, grid, candidates, k, scale):
+        """Head-aware tile search ("Head-Aware Tile Search"): for each candidate
+        tiling (applied to every head) the squared Frobenius distance between
+        full attention and the sparse layer output, per (candidate, b, h), and
+        per head the candidate with the smallest distance summed over b."""
+        Qb = _bf16_bits(Q)
+        B, H, N, d = Qb.shape
+        O_full, _ = self.full_attention(Q, K, V, grid, [candidates[0]] * H, scale)
+        err = np.empty((len(candidates), B, H))
+        for c, shape in enumerate(candidates):
+            shapes = [tuple(shape)] * H
+            r = self.mask_prep(Q, K, Wq, Wk, grid, shapes, k)
+            nT = r["idx"].shape[2]
+            O, lse, toks = self.sparse_attention(Q, K, V, r["idx"], grid, shapes, scale)
+            Oc, _ = self._scatter(O, lse, toks, B, H, N, d, nT)
+            err[c] = ((O_full - Oc) ** 2).sum(axis=(2, 3))
+        best = np.argmin(err.sum(axis=1), axis=0).astype(np.int32)  # first index on ties
+        return err, best, O_full

@@ -74,6 +74,7 @@ def pin_suite(o):
     yield lambda: pins.test_distill_gradient_matches_finite_differences(o, 0.7, 1)
     yield lambda: pins.test_distill_zero_when_target_equals_prediction(o)
     yield lambda: pins.test_distill_invariances_and_positivity(o)
+    yield lambda: pins.test_tile_search_brute_force(o)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -392,3 +392,33 @@ def test_distill_invariances_and_positivity(oracle):
     # S / tau is what matters: scaling Wq by 2 and tau by 2 leaves the loss unchanged
     L2 = oracle.distill_kl(sq, sk, (Wq * 2).astype(np.float32), Wk, T, 2.0, grads=False)
     assert abs(L2 - L) < 1e-12
+
+
+# ---------------------------------------------------------------- head-aware tile search
+def test_tile_search_brute_force(oracle):
+    grid, d, k = (2, 4, 8), 8, 2
+    cands = [(1, 2, 4), (2, 2, 2), (1, 4, 2)]
+    w, x, Wq, Wk = draw(grid, [cands[0], cands[0]], d, B=2)
+    scale = 1 / math.sqrt(d)
+    err, best, _ = oracle.tile_search(x["Q"], x["K"], x["V"], Wq, Wk, grid, cands, k, scale)
+    Qf, Kf, Vf = (bf.bits_to_f64(x[n]) for n in "QKV")
+    full = np.stack([np.stack([bf.masked_attention(Qf[b, h], Kf[b, h], Vf[b, h],
+                                                    np.ones((w.N, w.N), bool), scale)[0]
+                               for h in range(2)]) for b in range(2)])
+    for c, shape in enumerate(cands):
+        shapes = [shape, shape]
+        S = bf.scores(bf.tripool(Qf, grid, shapes), bf.tripool(Kf, grid, shapes), Wq, Wk)
+        mask, _ = bf.topk(S, k)
+        Os, _ = bf.sparse_attention(Qf, Kf, Vf, mask, grid, shapes, scale)
+        np.testing.assert_allclose(err[c], ((full - Os) ** 2).sum(axis=(2, 3)), rtol=1e-9,
+                                   atol=1e-12)
+    np.testing.assert_array_equal(best, np.argmin(err.sum(axis=1), axis=0))
+
+
+def test_tile_search_all_tiles_has_zero_error(oracle):
+    grid, d = (2, 4, 8), 8
+    cands = [(1, 2, 4), (2, 2, 2)]
+    w, x, Wq, Wk = draw(grid, [cands[0]], d)
+    err, best, _ = oracle.tile_search(x["Q"], x["K"], x["V"], Wq, Wk, grid, cands, 8, 0.3)
+    assert np.abs(err).max() < 1e-24
+    assert best.tolist() == [0]

@@ -81,6 +81,9 @@ def load_library(path: str = LIB_PATH):
     lib.veda_distill_kl.argtypes = ([ctypes.POINTER(veda_problem)] + [_P] * 6 + [ctypes.c_float]
                                     + [_P] * 4 + [_P])
     lib.veda_distill_kl.restype = st
+    lib.veda_tile_search.argtypes = ([ctypes.POINTER(veda_problem), _P, ctypes.c_int32]
+                                     + [_P] * 11)
+    lib.veda_tile_search.restype = st
     lib.veda_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.veda_tile_score_noalloc.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 6
     lib.veda_tile_score_noalloc.restype = st
@@ -231,6 +234,20 @@ def veda_distill_kl(problem: Problem, statsQ, statsK, Wq, Wk, S, teacher, tau, l
                                           _ptr(Wq), _ptr(Wk), _ptr(S), _ptr(teacher),
                                           ctypes.c_float(tau), _ptr(loss), _ptr(dWq), _ptr(dWk),
                                           _ptr(ws), _stream(stream)))
+
+
+def veda_tile_search(problem: Problem, candidates, Q, K, V, Wq, Wk, O_dense, O_cand, err, best,
+                     ws, stream=None) -> None:
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O_dense, "O_dense"), (O_cand, "O_cand")):
+        _expect(t, torch.bfloat16, n)
+    _expect(err, torch.float64, "err")
+    _expect(best, torch.int32, "best")
+    flat = [int(v) for c in candidates for v in c]
+    arr = (ctypes.c_int32 * len(flat))(*flat)
+    _check(load_library().veda_tile_search(ctypes.byref(problem.c), ctypes.cast(arr, _P),
+                                           len(candidates), _ptr(Q), _ptr(K), _ptr(V), _ptr(Wq),
+                                           _ptr(Wk), _ptr(O_dense), _ptr(O_cand), _ptr(err),
+                                           _ptr(best), _ptr(ws), _stream(stream)))
 
 
 def veda_get_status(ws, stream=None) -> int:

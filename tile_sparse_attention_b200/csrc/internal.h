@@ -90,6 +90,17 @@ veda_status launch_distill(const Problem& pr, const float* statsQ, const float* 
                            float tau, double* loss, float* dWq, float* dWk, void* ws,
                            cudaStream_t s);
 
+// Head-aware tile search helpers (tile_search.cu).
+veda_status launch_sq_err(const uint16_t* a, const uint16_t* b, int heads, long long per_head,
+                          double* err, cudaStream_t s);
+veda_status launch_argmin(const double* err, int ncand, int B, int H, int32_t* best,
+                          cudaStream_t s);
+// The whole layer on a validated problem (veda_api.cu).
+veda_status forward_impl(const Problem& pr, const uint16_t* Q, const uint16_t* K,
+                         const uint16_t* V, const float* Wq, const float* Wk, uint16_t* O,
+                         float* lse, int32_t* idx_out, uint8_t* mask_out, void* ws,
+                         cudaStream_t s);
+
 // Workspace layout of veda_forward (byte offsets, 256-aligned).
 struct WorkspaceLayout {
     size_t status, statsQ, statsK, qt, kt, S, idx, total;

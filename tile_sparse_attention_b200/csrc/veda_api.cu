@@ -123,6 +123,29 @@ WorkspaceLayout workspace_layout(const Problem& pr) {
     return w;
 }
 
+// The layer on an already validated problem; the status word in ws is not cleared.
+veda_status forward_impl(const Problem& pr, const uint16_t* Q, const uint16_t* K,
+                         const uint16_t* V, const float* Wq, const float* Wk, uint16_t* O,
+                         float* lse, int32_t* idx_out, uint8_t* mask_out, void* ws,
+                         cudaStream_t s) {
+    const WorkspaceLayout w = workspace_layout(pr);
+    char* base = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(base + w.status);
+    float* statsQ = reinterpret_cast<float*>(base + w.statsQ);
+    float* statsK = reinterpret_cast<float*>(base + w.statsK);
+    float* qt = reinterpret_cast<float*>(base + w.qt);
+    float* kt = reinterpret_cast<float*>(base + w.kt);
+    float* S = reinterpret_cast<float*>(base + w.S);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+    veda_status st;
+    if ((st = launch_tripool(pr, Q, K, statsQ, statsK, s))) return st;
+    if ((st = launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
+    if ((st = launch_project(pr, statsK, Wk, kt, 1, s))) return st;
+    if ((st = launch_score(pr, qt, kt, S, status, s))) return st;
+    if ((st = launch_topk(pr, S, mask_out, idx, s))) return st;
+    return launch_sparse_attn(pr, Q, K, V, idx, pr.k, O, lse, status, s);
+}
+
 }  // namespace veda
 
 using namespace veda;
@@ -216,22 +239,54 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
         (st = check_ptr(mask_out, "mask_out", true)) || (st = check_ptr(ws, "ws")))
         return st;
     cudaStream_t s = (cudaStream_t)stream;
-    const WorkspaceLayout w = workspace_layout(pr);
-    char* base = static_cast<char*>(ws);
-    int* status = reinterpret_cast<int*>(base + w.status);
-    float* statsQ = reinterpret_cast<float*>(base + w.statsQ);
-    float* statsK = reinterpret_cast<float*>(base + w.statsK);
-    float* qt = reinterpret_cast<float*>(base + w.qt);
-    float* kt = reinterpret_cast<float*>(base + w.kt);
-    float* S = reinterpret_cast<float*>(base + w.S);
-    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+    if ((st = cuda_check(cudaMemsetAsync(ws, 0, sizeof(int), s), "status reset"))) return st;
+    return forward_impl(pr, Q, K, V, Wq, Wk, O, lse, idx_out, mask_out, ws, s);
+}
+
+veda_status veda_tile_search(const veda_problem* p, const int32_t* candidates, int32_t ncand,
+                             const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                             const float* Wq, const float* Wk, uint16_t* O_dense,
+                             uint16_t* O_cand, double* err, int32_t* best, void* ws,
+                             veda_stream_t stream) {
+    if (p == nullptr || candidates == nullptr)
+        return fail(VEDA_ERR_INVALID_ARG, "problem and candidates must be non-NULL");
+    if (ncand < 1 || ncand > 16) return fail(VEDA_ERR_INVALID_ARG, "1 to 16 candidate tilings");
+    if (p->H < 1 || p->H > kMaxHeads) return fail(VEDA_ERR_UNSUPPORTED, "at most 256 heads");
+    veda_status st;
+    if ((st = check_ptr(Q, "Q")) || (st = check_ptr(K, "K")) || (st = check_ptr(V, "V")) ||
+        (st = check_ptr(Wq, "Wq")) || (st = check_ptr(Wk, "Wk")) ||
+        (st = check_ptr(O_dense, "O_dense")) || (st = check_ptr(O_cand, "O_cand")) ||
+        (st = check_ptr(err, "err")) || (st = check_ptr(best, "best")) || (st = check_ptr(ws, "ws")))
+        return st;
+    // every candidate tiling, applied to every head, must make a valid problem
+    // with the same tile count
+    static thread_local int32_t shapes[16][kMaxHeads * 3];
+    Problem prs[16];
+    for (int c = 0; c < ncand; ++c) {
+        for (int h = 0; h < p->H; ++h)
+            for (int q = 0; q < 3; ++q) shapes[c][3 * h + q] = candidates[3 * c + q];
+        veda_problem pc = *p;
+        pc.tile_shapes = shapes[c];
+        if ((st = make_problem(&pc, true, &prs[c])) != VEDA_OK) return st;
+        if (prs[c].nT != prs[0].nT)
+            return fail(VEDA_ERR_SHAPE, "candidate tilings must have the same tile size");
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    int* status = static_cast<int*>(ws);
     if ((st = cuda_check(cudaMemsetAsync(status, 0, sizeof(int), s), "status reset"))) return st;
-    if ((st = launch_tripool(pr, Q, K, statsQ, statsK, s))) return st;
-    if ((st = launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
-    if ((st = launch_project(pr, statsK, Wk, kt, 1, s))) return st;
-    if ((st = launch_score(pr, qt, kt, S, status, s))) return st;
-    if ((st = launch_topk(pr, S, mask_out, idx, s))) return st;
-    return launch_sparse_attn(pr, Q, K, V, idx, pr.k, O, lse, status, s);
+    const Problem& p0 = prs[0];
+    // full attention (the dense schedule does not depend on the tiling)
+    if ((st = launch_sparse_attn(p0, Q, K, V, nullptr, p0.nT, O_dense, nullptr, status, s)))
+        return st;
+    const long long per_head = (long long)p0.N * p0.d;
+    for (int c = 0; c < ncand; ++c) {
+        if ((st = forward_impl(prs[c], Q, K, V, Wq, Wk, O_cand, nullptr, nullptr, nullptr, ws, s)))
+            return st;
+        if ((st = launch_sq_err(O_dense, O_cand, p0.B * p0.H, per_head,
+                                err + (size_t)c * p0.B * p0.H, s)))
+            return st;
+    }
+    return launch_argmin(err, ncand, p0.B, p0.H, best, s);
 }
 
 veda_status veda_teacher(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
