@@ -41,6 +41,13 @@ import workloads  # noqa: E402
 METRIC = "ms/layer and effective TFLOP/s of tile-sparse attention (+mask prep) at 95% sparsity"
 
 
+# DRAM bytes (read + write) of one attention launch, from one ncu capture of
+# dram__bytes_read.sum + dram__bytes_write.sum on this kernel version (profile
+# summary: profiles/launches_long_video_245k.md).  Emptied whenever the kernel
+# changes, until the counters are taken again.
+ATTN_DRAM_BYTES = {"long_video_245k": 3.41e9 + 2.02e9}
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -77,6 +84,12 @@ def _max_over_ranks(x: float, world: int) -> float:
     t = torch.tensor([x], dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def _job_tflops(flops_per_replica: float, ms_per_step_max: float, world: int) -> float:
+    """Whole-job throughput: every rank runs one replica of the layer per step,
+    so the job does world x the work in the slowest rank's time."""
+    return world * flops_per_replica / (ms_per_step_max * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------- clocks
@@ -162,7 +175,8 @@ def oracle_sample(w, t_host, heads=1, units_per_head=24, threads=None):
     t1 = time.perf_counter()
     rng = np.random.default_rng(0)
     units = np.array([(0, h, int(i)) for h in range(heads)
-                      for i in rng.choice(w.nT, units_per_head, replace=False)], dtype=np.int64)
+                      for i in rng.choice(w.nT, min(units_per_head, w.nT), replace=False)],
+                     dtype=np.int64)
     o.sparse_attention(Qb, Kb, Vb, r["idx"], w.grid, shapes, w.scale, units=units)
     t2 = time.perf_counter()
     prep_per_head = (t1 - t0) / heads
@@ -269,7 +283,7 @@ def run_veda(args, w, world, rank, local):
     per = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
            for i, n in enumerate(["tripool", "tile_score", "topk", "sparse_attn"])}
     flops = w.sparse_flops()
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = _job_tflops(flops, ms, world)
 
     # mask-prep kernels as a fraction of HBM bandwidth (algorithmic bytes)
     tri_bytes = 2 * B * H * N * d * 2 + 2 * B * H * nT * 3 * d * 4
@@ -336,7 +350,7 @@ def run_veda(args, w, world, rank, local):
         _barrier(world)
         e_ms = _max_over_ranks(a.elapsed_time(b) / n_e2e, world)
         h2d = sum(x.numel() * x.element_size() for x in (hostQ, hostK, hostV, hostWq, hostWk))
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": _job_tflops(flops, e_ms, world), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": hostO.numel() * hostO.element_size()}
         del hostQ, hostK, hostV, hostO, dQ, dK, dV
@@ -346,7 +360,8 @@ def run_veda(args, w, world, rank, local):
         th = {n: workloads.bf16_bits(t[n].index_select(1, torch.tensor([0], device=dev)))
               for n in ("Q", "K", "V")}
         th["Wq"], th["Wk"] = t["Wq"].cpu().numpy(), t["Wk"].cpu().numpy()
-        res = oracle_sample(w, th, heads=1, units_per_head=24)
+        # about 10-15 s of fp64 work on the host cores at the long-video size
+        res = oracle_sample(w, th, heads=1, units_per_head=512)
         cpu = {"value": flops / res["full_layer_s"] / 1e12, "unit": "TFLOP/s",
                "cores": res["cores"], "kind": "oracle", "sample": res["sample"],
                "seconds_sampled": res["seconds_sampled"],
@@ -370,7 +385,8 @@ def run_veda(args, w, world, rank, local):
             "roofline": {"bound": "tensor", "kernel": "sparse_attn", "achieved": attn_tf,
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
                          "peak_kind": "bf16 sustained (" + peaks["source"] + ")",
-                         "frac_of_burst": attn_tf / peaks["bf16"], "traffic": None,
+                         "frac_of_burst": attn_tf / peaks["bf16"],
+                         "traffic": ATTN_DRAM_BYTES.get(w.name),
                          "algorithmic_flops_per_launch": flops},
             "kernels_ms": per,
             "mask_prep": mask_prep,

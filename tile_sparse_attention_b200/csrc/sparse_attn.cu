@@ -67,6 +67,7 @@ struct __align__(64) AttnParams {
     int H, T, Hs, Ws, N, nT, k;
     float scale_log2;
     unsigned long long wait_limit_ns;
+    int withhold_arrive;  // failure-detection test only: warp 4 skips its first P-ready arrival
 };
 
 template <int D, int BT, int NS>
@@ -437,7 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
+            if (lane == 0 && !(p.withhold_arrive && j == 0 && wq == 0))
+                mbar_arrive(&bars.p_full[j & 1]);
         }
         if (ok) ok = warp_wait_bar(&bars.kv_empty[(k - 1) % NS], ((k - 1) / NS) & 1, p, abort_flag);
         // every softmax thread gets here (all waits are bounded); the epilogue
@@ -537,6 +539,10 @@ veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint1
     prm.k = k;
     prm.scale_log2 = pr.scale * 1.4426950408889634f;
     prm.wait_limit_ns = wait_limit_ns();
+    // Test hook for the bounded waits: with VEDA_TEST_WITHHOLD_ARRIVE set, one
+    // arrival never happens, the MMA issuer's wait runs out and every CTA
+    // reports VEDA_ERR_TIMEOUT (nothing in normal use sets the variable).
+    prm.withhold_arrive = getenv("VEDA_TEST_WITHHOLD_ARRIVE") != nullptr ? 1 : 0;
     if (pr.d == 128 && pr.Bt == 128) return launch_cfg<128, 128, 3>(prm, pr, s);
     if (pr.d == 128 && pr.Bt == 64) return launch_cfg<128, 64, 4>(prm, pr, s);
     if (pr.d == 64 && pr.Bt == 128) return launch_cfg<64, 128, 4>(prm, pr, s);
