@@ -124,6 +124,26 @@ veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask,
                            veda_stream_t stream);
 
 /*
+ * Fused tile score + head-aware Top-k (project page, "Attention Structure
+ * Distillation", Estimator and Execution): the same projection, score and
+ * selection as veda_tile_score followed by veda_topk_mask, with the score
+ * matrix S held on chip (never written to memory).  Results are identical to
+ * the two-call path (the scores are computed by the same products in the same
+ * order).
+ *   statsQ, statsK, Wq, Wk: as for veda_tile_score
+ *   mask: uint8 [B, H, nT, nT] of 0/1, may be NULL
+ *   idx : int32 [B, H, nT, k], the kept tile indices in ascending order
+ *   ws  : device workspace of at least VEDA_STATUS_BYTES + 2 * B*H*nT*9*d*4
+ *         bytes (the projected statistics); veda_workspace_size() is enough.
+ * Limits: k <= 128 and nT <= 6144, else VEDA_ERR_UNSUPPORTED (use the two-call
+ * path).  A device-side wait that gives up is reported through
+ * veda_get_status(ws) as VEDA_ERR_TIMEOUT.
+ */
+veda_status veda_mask_fused(const veda_problem* p, const float* statsQ, const float* statsK,
+                            const float* Wq, const float* Wk, uint8_t* mask, int32_t* idx,
+                            void* ws, veda_stream_t stream);
+
+/*
  * Tile-skipping attention (project page, "Attention Structure Distillation",
  * Execution and "Principle 03 Tile-Sparse Kernel"; "Theoretical Rationale" 1:
  * the kept keys are renormalised among themselves).  For every query token of

@@ -65,6 +65,8 @@ def load_library(path: str = LIB_PATH):
     lib.veda_tile_score.restype = st
     lib.veda_topk_mask.argtypes = [ctypes.POINTER(veda_problem), _P, _P, _P, _P]
     lib.veda_topk_mask.restype = st
+    lib.veda_mask_fused.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 8
+    lib.veda_mask_fused.restype = st
     lib.veda_sparse_attn.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 8
     lib.veda_sparse_attn.restype = st
     lib.veda_forward.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 11
@@ -172,6 +174,17 @@ def veda_topk_mask(problem: Problem, S, mask, idx, stream=None) -> None:
     _expect(idx, torch.int32, "idx")
     _check(load_library().veda_topk_mask(ctypes.byref(problem.c), _ptr(S), _ptr(mask), _ptr(idx),
                                          _stream(stream)))
+
+
+def veda_mask_fused(problem: Problem, statsQ, statsK, Wq, Wk, mask, idx, ws, stream=None) -> None:
+    for t, n in ((statsQ, "statsQ"), (statsK, "statsK"), (Wq, "Wq"), (Wk, "Wk")):
+        _expect(t, torch.float32, n)
+    _expect(idx, torch.int32, "idx")
+    if mask is not None:
+        _expect(mask, torch.uint8, "mask")
+    _check(load_library().veda_mask_fused(ctypes.byref(problem.c), _ptr(statsQ), _ptr(statsK),
+                                          _ptr(Wq), _ptr(Wk), _ptr(mask), _ptr(idx), _ptr(ws),
+                                          _stream(stream)))
 
 
 def veda_sparse_attn(problem: Problem, Q, K, V, idx, O, lse, ws, stream=None) -> None:

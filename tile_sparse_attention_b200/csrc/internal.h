@@ -49,6 +49,10 @@ veda_status launch_score(const Problem& pr, const float* qext, const float* kext
 inline size_t projected_bytes(const Problem& pr) {
     return (size_t)pr.B * pr.H * pr.nT * 9 * pr.d * sizeof(float);
 }
+// Fused score + Top-k (S stays on chip); needs k <= 128 and nT <= 6144.
+bool fused_mask_supported(const Problem& pr);
+veda_status launch_score_topk(const Problem& pr, const float* qext, const float* kext,
+                              uint8_t* mask, int32_t* idx, int* status, cudaStream_t s);
 veda_status launch_topk(const Problem& pr, const float* S, uint8_t* mask, int32_t* idx,
                         cudaStream_t s);
 veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint16_t* K,

@@ -209,6 +209,30 @@ veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask,
     return launch_topk(pr, S, mask, idx, (cudaStream_t)stream);
 }
 
+veda_status veda_mask_fused(const veda_problem* p, const float* statsQ, const float* statsK,
+                            const float* Wq, const float* Wk, uint8_t* mask, int32_t* idx,
+                            void* ws, veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, true, &pr)) != VEDA_OK) return st;
+    if ((st = check_ptr(statsQ, "statsQ")) || (st = check_ptr(statsK, "statsK")) ||
+        (st = check_ptr(Wq, "Wq")) || (st = check_ptr(Wk, "Wk")) || (st = check_ptr(idx, "idx")) ||
+        (st = check_ptr(mask, "mask", true)) || (st = check_ptr(ws, "ws")))
+        return st;
+    if (!fused_mask_supported(pr))
+        return fail(VEDA_ERR_UNSUPPORTED, "fused mask: needs k <= 128 and nT <= 6144");
+    cudaStream_t s = (cudaStream_t)stream;
+    const WorkspaceLayout w = workspace_layout(pr);
+    char* base = static_cast<char*>(ws);
+    float* qt = reinterpret_cast<float*>(base + w.qt);
+    float* kt = reinterpret_cast<float*>(base + w.kt);
+    int* status = reinterpret_cast<int*>(base + w.status);
+    if ((st = cuda_check(cudaMemsetAsync(status, 0, sizeof(int), s), "status reset"))) return st;
+    if ((st = launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
+    if ((st = launch_project(pr, statsK, Wk, kt, 1, s))) return st;
+    return launch_score_topk(pr, qt, kt, mask, idx, status, s);
+}
+
 veda_status veda_sparse_attn(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
                              const uint16_t* V, const int32_t* idx, uint16_t* O, float* lse,
                              void* ws, veda_stream_t stream) {
