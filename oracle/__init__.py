@@ -60,6 +60,12 @@ def _bind(lib):
     lib.oracle_tile_recall.restype = ctypes.c_double
     lib.oracle_distill_kl.argtypes = [_I64] * 4 + [_P] * 5 + [ctypes.c_double, _P, _P]
     lib.oracle_distill_kl.restype = ctypes.c_double
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_int32]
+    lib.oracle_e4m3_decode.restype = ctypes.c_double
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_encode.restype = ctypes.c_int32
+    lib.oracle_quantize_e4m3.argtypes = [_I64, _I64, _P, _P, _P]
+    lib.oracle_dequantize_e4m3.argtypes = [_I64, _I64, _P, _P, _P]
     return lib
 
 
@@ -225,6 +231,34 @@ class Oracle:
                                           _ptr(dWq) if grads else None,
                                           _ptr(dWk) if grads else None)
         return (float(loss), dWq, dWk) if grads else float(loss)
+
+    def e4m3_decode(self, code: int) -> float:
+        """Value of an fp8 E4M3 code (NaN for 0x7F / 0xFF)."""
+        return float(self.lib.oracle_e4m3_decode(int(code)))
+
+    def e4m3_encode(self, x: float) -> int:
+        """Nearest E4M3 code of an fp32 value (ties to the even code, saturating)."""
+        return int(self.lib.oracle_e4m3_encode(float(np.float32(x))))
+
+    def quantize_e4m3(self, W):
+        """Per-head fp8 E4M3 weights: codes uint8 [H, ...] and fp32 scale [H]."""
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        H = W.shape[0]
+        n = W.size // H
+        codes = np.empty(W.shape, dtype=np.uint8)
+        scale = np.empty((H,), dtype=np.float32)
+        self.lib.oracle_quantize_e4m3(H, n, _ptr(W), _ptr(codes), _ptr(scale))
+        return codes, scale
+
+    def dequantize_e4m3(self, codes, scale):
+        """fp32 weights e4m3(code) * scale[h]."""
+        codes = np.ascontiguousarray(codes, dtype=np.uint8)
+        scale = np.ascontiguousarray(scale, dtype=np.float32)
+        H = codes.shape[0]
+        n = codes.size // H
+        W = np.empty(codes.shape, dtype=np.float32)
+        self.lib.oracle_dequantize_e4m3(H, n, _ptr(codes), _ptr(scale), _ptr(W))
+        return W
 
     def full_attention(self, Q, K, V, grid, tile_shapes, scale):
         """Dense softmax attention for every token: O [B,H,N,d] fp64, lse [B,H,N]."""

@@ -477,3 +477,88 @@ double oracle_distill_kl(int64_t B, int64_t H, int64_t nT, int64_t d,
     free(G);
     return total / (double)R;
 }
+
+/* ----------------------------------------------------------- fp8 weights
+ * fp8 estimator weights.  News page ("Veda from ByteDance, HKU and USTC: an
+ * open method that speeds up video generation fivefold", "Why this matters
+ * for users"): the predictor is distributed in fp8 at half the size of the
+ * bf16 file with almost the same tile recall.  The page names no encoding or
+ * scaling; the reading taken here is the OCP FP8 E4M3 format ("e4m3fn": 1
+ * sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no infinities; the
+ * all-ones exponent with all-ones mantissa is NaN, so the largest finite
+ * value is 1.75 * 2^8 = 448; exponent field 0 holds the subnormals
+ * m/8 * 2^-6) with one scale per head, s = amax / 448, W ~= s * e4m3(W / s),
+ * rounding to the nearest code, ties to the even code, saturating at +-448.
+ * The scale and W / s are fp32 operations (the quantiser's decisions are
+ * taken on fp32 values); the dequantised weight is the fp32 product
+ * e4m3 * s, the weight the fp32 estimator then computes with.
+ */
+double oracle_e4m3_decode(int32_t code)
+{
+    const int sign = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest e4m3 code of an fp32 value: ties to the even code, saturating. */
+int32_t oracle_e4m3_encode(float x)
+{
+    if (isnan(x)) return 0x7F;
+    const int32_t sign = signbit(x) ? 0x80 : 0;
+    const double a = fabs((double)x);
+    if (a >= 448.0) return sign | 126;
+    /* codes 0..126 are the non-negative finite values in increasing order:
+       find the largest code whose value is <= a */
+    int32_t lo = 0, hi = 126;
+    while (lo < hi) {
+        const int32_t mid = (lo + hi + 1) / 2;
+        if (oracle_e4m3_decode(mid) <= a)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const double dlo = a - oracle_e4m3_decode(lo);      /* exact in fp64 */
+    const double dhi = oracle_e4m3_decode(lo + 1) - a;
+    int32_t code;
+    if (dlo < dhi)
+        code = lo;
+    else if (dlo > dhi)
+        code = lo + 1;
+    else
+        code = (lo & 1) ? lo + 1 : lo;
+    return sign | code;
+}
+
+/* W: fp32 [H][n]; codes: uint8 [H][n]; scale: fp32 [H]. */
+void oracle_quantize_e4m3(int64_t H, int64_t n, const float* W, uint8_t* codes, float* scale)
+{
+    for (int64_t h = 0; h < H; ++h) {
+        float amax = 0.0f;
+        for (int64_t i = 0; i < n; ++i) {
+            const float a = fabsf(W[h * n + i]);
+            if (a > amax) amax = a;
+        }
+        const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[h] = s;
+        for (int64_t i = 0; i < n; ++i) {
+            const float y = W[h * n + i] / s;
+            codes[h * n + i] = (uint8_t)oracle_e4m3_encode(y);
+        }
+    }
+}
+
+/* W[h][i] = fp32(e4m3(codes[h][i]) * scale[h]). */
+void oracle_dequantize_e4m3(int64_t H, int64_t n, const uint8_t* codes, const float* scale,
+                            float* W)
+{
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t i = 0; i < n; ++i) {
+            const float v = (float)oracle_e4m3_decode(codes[h * n + i]);
+            W[h * n + i] = v * scale[h];
+        }
+}

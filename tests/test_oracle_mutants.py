@@ -47,6 +47,10 @@ MUTANTS = {
         "dWq[(h * d + ci) * d + co] += sq[ci] * dq[s3 * d + co];",
         "dWq[(h * d + ci) * d + co] += sk[ci] * dq[s3 * d + co];"),
     "distillation target not normalised": ("double tg = t[j] / tsum;", "double tg = t[j];"),
+    "e4m3 ties go to the lower code": ("code = (lo & 1) ? lo + 1 : lo;", "code = lo;"),
+    "e4m3 exponent bias 8": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+                             "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3 scale from the mean magnitude": ("if (a > amax) amax = a;", "amax += a / (float)n;"),
 }
 
 
@@ -75,6 +79,9 @@ def pin_suite(o):
     yield lambda: pins.test_distill_zero_when_target_equals_prediction(o)
     yield lambda: pins.test_distill_invariances_and_positivity(o)
     yield lambda: pins.test_tile_search_brute_force(o)
+    yield lambda: pins.test_e4m3_format_facts(o)
+    yield lambda: pins.test_e4m3_round_trip_midpoints_and_saturation(o)
+    yield lambda: pins.test_e4m3_quantize_per_head(o)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -422,3 +422,75 @@ def test_tile_search_all_tiles_has_zero_error(oracle):
     err, best, _ = oracle.tile_search(x["Q"], x["K"], x["V"], Wq, Wk, grid, cands, 8, 0.3)
     assert np.abs(err).max() < 1e-24
     assert best.tolist() == [0]
+
+
+# ------------------------------------------------------------------ fp8 weights
+# OCP FP8 E4M3 ("e4m3fn") format facts: bias 7, 3 mantissa bits, no infinities,
+# S.1111.111 is NaN, largest finite 1.75 * 2^8 = 448, smallest normal 2^-6,
+# smallest subnormal 2^-9.
+def test_e4m3_format_facts(oracle):
+    o = oracle
+    assert o.e4m3_decode(0x7E) == 448.0 and o.e4m3_decode(0xFE) == -448.0
+    assert np.isnan(o.e4m3_decode(0x7F)) and np.isnan(o.e4m3_decode(0xFF))
+    assert o.e4m3_decode(0x08) == 2.0 ** -6 and o.e4m3_decode(0x07) == 7 * 2.0 ** -9
+    assert o.e4m3_decode(0x01) == 2.0 ** -9
+    assert o.e4m3_decode(0x38) == 1.0 and o.e4m3_decode(0x3C) == 1.5
+    z = o.e4m3_decode(0x80)
+    assert z == 0.0 and np.signbit(z)
+    vals = [o.e4m3_decode(c) for c in range(127)]
+    assert all(b > a for a, b in zip(vals, vals[1:]))
+
+
+def test_e4m3_round_trip_midpoints_and_saturation(oracle):
+    o = oracle
+    for c in list(range(127)) + list(range(128, 255)):
+        assert o.e4m3_encode(o.e4m3_decode(c)) == c
+    for c in range(126):
+        a, b = o.e4m3_decode(c), o.e4m3_decode(c + 1)
+        mid = np.float32((a + b) / 2)          # one extra bit: exact in fp32
+        assert float(mid) == (a + b) / 2
+        even = c if c % 2 == 0 else c + 1
+        assert o.e4m3_encode(mid) == even
+        assert o.e4m3_encode(-mid) == 0x80 | even
+        assert o.e4m3_encode(np.nextafter(mid, np.float32(0))) == c
+        assert o.e4m3_encode(np.nextafter(mid, np.float32(1000))) == c + 1
+    for x in (448.0, 449.0, 463.9, 464.0, 1e4, 3e38):
+        assert o.e4m3_encode(x) == 0x7E and o.e4m3_encode(-x) == 0xFE
+
+
+def test_e4m3_matches_library_conversion(oracle):
+    """Round to nearest even, as torch's float8_e4m3fn conversion does (|x| <= 448)."""
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.uniform(-448, 448, 4000), rng.standard_normal(4000),
+                        rng.standard_normal(2000) * 2.0 ** -7,
+                        rng.standard_normal(1000) * 2.0 ** -10]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(v) for v in x], dtype=np.uint8)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_e4m3_quantize_per_head(oracle):
+    rng = np.random.default_rng(12)
+    W = (rng.standard_normal((4, 16, 16)) / 4).astype(np.float32)
+    W[1] *= 1e-3                               # small values, subnormal codes
+    W[2] = 0.0                                 # all-zero head: scale 1, zero codes
+    W[3, 5, 7] = -7.5                          # a single large value sets the scale
+    codes, scale = oracle.quantize_e4m3(W)
+    for h in range(4):
+        amax = np.abs(W[h]).max()
+        want = np.float32(amax) / np.float32(448.0) if amax > 0 else np.float32(1.0)
+        assert scale[h] == want
+    assert np.all(codes[2] == 0)
+    assert codes[3, 5, 7] == 0xFE
+    Wd = oracle.dequantize_e4m3(codes, scale)
+    assert Wd.dtype == np.float32 and Wd[3, 5, 7] == np.float32(np.float32(-448.0) * scale[3])
+    for h in (0, 1, 3):
+        s = float(scale[h])
+        y = np.abs(W[h].astype(np.float64)) / s
+        # half a code step: 2^(e-4) in a normal binade, 2^-10 below 2^-6; plus fp32 rounding
+        step = np.where(y >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(y, 1e-30))) - 4), 2.0 ** -10)
+        err = np.abs(Wd[h].astype(np.float64) - W[h].astype(np.float64))
+        assert np.all(err <= s * step * (1 + 2.0 ** -20) + np.abs(W[h]) * 2.0 ** -23)
+    # decoding the codes by the format definition gives the same weights
+    dec = np.vectorize(oracle.e4m3_decode)(codes.astype(np.int64)).astype(np.float32)
+    np.testing.assert_array_equal(Wd, (dec * scale[:, None, None]).astype(np.float32))
