@@ -481,6 +481,40 @@ def run_rows(args, w, rows):
         print(json.dumps({"row": "f2 head-aware tile search", "workload": w.name,
                           "candidates": cands, "ms": ms, "heads_per_candidate": picks,
                           "status": vb.veda_get_status(ws)}), flush=True)
+    if "f4" in rows:
+        statsQ = torch.empty((B, H, nT, 3, d), dtype=torch.float32, device=dev)
+        statsK = torch.empty_like(statsQ)
+        vb.veda_tripool(prob, t["Q"], t["K"], statsQ, statsK)
+        S = torch.empty((B, H, nT, nT), dtype=torch.float32, device=dev)
+        idx2 = torch.empty((B, H, nT, k), dtype=torch.int32, device=dev)
+        idxf = torch.empty_like(idx2)
+        ms_two = timed(lambda: (vb.veda_tile_score(prob, statsQ, statsK, t["Wq"], t["Wk"], S, ws),
+                                vb.veda_topk_mask(prob, S, None, idx2)), reps=10)
+        ms_fused = timed(lambda: vb.veda_mask_fused(prob, statsQ, statsK, t["Wq"], t["Wk"], None,
+                                                    idxf, ws), reps=10)
+        same = bool(torch.equal(idx2, idxf))
+        # fp8 (E4M3) estimator weights: quantise, dequantise, mask, recall vs fp32
+        W8 = torch.empty((H, d, d), dtype=torch.uint8, device=dev)
+        sc = torch.empty((H,), dtype=torch.float32, device=dev)
+        deq = {}
+        for name in ("Wq", "Wk"):
+            vb.veda_quantize_fp8(t[name], W8, sc)
+            deq[name] = torch.empty_like(t[name])
+            vb.veda_dequantize_fp8(W8, sc, deq[name])
+        ms_q = timed(lambda: vb.veda_quantize_fp8(t["Wq"], W8, sc), reps=10)
+        ms_dq = timed(lambda: vb.veda_dequantize_fp8(W8, sc, deq["Wq"]), reps=10)
+        idx8 = torch.empty_like(idx2)
+        vb.veda_mask_fused(prob, statsQ, statsK, deq["Wq"], deq["Wk"], None, idx8, ws)
+        mean = torch.empty((1,), dtype=torch.float64, device=dev)
+        vb.veda_tile_recall(prob, idx8, idxf, None, mean, ws)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"row": "f4 fused mask prep + fp8 estimator weights", "workload": w.name,
+                          "score_plus_topk_ms": ms_two, "fused_mask_ms": ms_fused,
+                          "fused_equals_two_call": same, "S_bytes_not_written": S.numel() * 4,
+                          "fp8_quantize_ms": ms_q, "fp8_dequantize_ms": ms_dq,
+                          "weight_bytes_fp32": 2 * H * d * d * 4, "weight_bytes_fp8": 2 * H * (d * d + 4),
+                          "tile_recall_fp8_vs_fp32_mask": mean.item(),
+                          "status": vb.veda_get_status(ws)}), flush=True)
     return 0
 
 
@@ -496,7 +530,7 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--rows", default="",
-                    help="comma list of f1,f2,f3: time the training-side rows instead")
+                    help="comma list of f1,f2,f3,f4: time the next rows instead")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "veda":
         args.warmup = 3

@@ -124,6 +124,23 @@ veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask,
                            veda_stream_t stream);
 
 /*
+ * fp8 estimator weights (news page "Veda from ByteDance, HKU and USTC: an open
+ * method that speeds up video generation fivefold", "Why this matters for
+ * users": the predictor is distributed in fp8).  Encoding: OCP FP8 E4M3, one
+ * scale per head:
+ *   scale[h] = max |W[h]| / 448 (fp32; 1 for an all-zero head),
+ *   W8[h]    = E4M3(W[h] / scale[h]), round to nearest even, saturating at +-448.
+ *   W    : fp32 [H, d, d] (device)      W8: uint8 [H, d, d]      scale: fp32 [H]
+ * veda_dequantize_fp8 writes the fp32 weights fp32(E4M3(W8) * scale[h]), which
+ * veda_tile_score / veda_mask_fused / veda_forward take as Wq, Wk.
+ * Errors: VEDA_ERR_INVALID_ARG (H < 1, d < 1 or a NULL pointer).
+ */
+veda_status veda_quantize_fp8(const float* W, int64_t H, int64_t d, uint8_t* W8, float* scale,
+                              veda_stream_t stream);
+veda_status veda_dequantize_fp8(const uint8_t* W8, const float* scale, int64_t H, int64_t d,
+                                float* W, veda_stream_t stream);
+
+/*
  * Fused tile score + head-aware Top-k (project page, "Attention Structure
  * Distillation", Estimator and Execution): the same projection, score and
  * selection as veda_tile_score followed by veda_topk_mask, with the score

@@ -65,6 +65,10 @@ def load_library(path: str = LIB_PATH):
     lib.veda_tile_score.restype = st
     lib.veda_topk_mask.argtypes = [ctypes.POINTER(veda_problem), _P, _P, _P, _P]
     lib.veda_topk_mask.restype = st
+    lib.veda_quantize_fp8.argtypes = [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P]
+    lib.veda_quantize_fp8.restype = st
+    lib.veda_dequantize_fp8.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int64, _P, _P]
+    lib.veda_dequantize_fp8.restype = st
     lib.veda_mask_fused.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 8
     lib.veda_mask_fused.restype = st
     lib.veda_sparse_attn.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 8
@@ -174,6 +178,25 @@ def veda_topk_mask(problem: Problem, S, mask, idx, stream=None) -> None:
     _expect(idx, torch.int32, "idx")
     _check(load_library().veda_topk_mask(ctypes.byref(problem.c), _ptr(S), _ptr(mask), _ptr(idx),
                                          _stream(stream)))
+
+
+def veda_quantize_fp8(W, W8, scale, stream=None) -> None:
+    """W fp32 [H, d, d] -> W8 uint8 [H, d, d] (E4M3 codes), scale fp32 [H]."""
+    _expect(W, torch.float32, "W")
+    _expect(W8, torch.uint8, "W8")
+    _expect(scale, torch.float32, "scale")
+    H, d = W.shape[0], W.shape[-1]
+    _check(load_library().veda_quantize_fp8(_ptr(W), H, d, _ptr(W8), _ptr(scale), _stream(stream)))
+
+
+def veda_dequantize_fp8(W8, scale, W, stream=None) -> None:
+    """W8 uint8 [H, d, d], scale fp32 [H] -> W fp32 [H, d, d]."""
+    _expect(W8, torch.uint8, "W8")
+    _expect(scale, torch.float32, "scale")
+    _expect(W, torch.float32, "W")
+    H, d = W8.shape[0], W8.shape[-1]
+    _check(load_library().veda_dequantize_fp8(_ptr(W8), _ptr(scale), H, d, _ptr(W),
+                                              _stream(stream)))
 
 
 def veda_mask_fused(problem: Problem, statsQ, statsK, Wq, Wk, mask, idx, ws, stream=None) -> None:

@@ -49,6 +49,11 @@ veda_status launch_score(const Problem& pr, const float* qext, const float* kext
 inline size_t projected_bytes(const Problem& pr) {
     return (size_t)pr.B * pr.H * pr.nT * 9 * pr.d * sizeof(float);
 }
+// fp8 (E4M3) weights, one scale per head: W [H][n] fp32 <-> codes [H][n], scale [H].
+veda_status launch_quantize_e4m3(const float* W, int H, long long n, uint8_t* codes, float* scale,
+                                 cudaStream_t s);
+veda_status launch_dequantize_e4m3(const uint8_t* codes, const float* scale, int H, long long n,
+                                   float* W, cudaStream_t s);
 // Fused score + Top-k (S stays on chip); needs k <= 128 and nT <= 6144.
 bool fused_mask_supported(const Problem& pr);
 veda_status launch_score_topk(const Problem& pr, const float* qext, const float* kext,

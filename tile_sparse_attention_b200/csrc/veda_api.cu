@@ -209,6 +209,26 @@ veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask,
     return launch_topk(pr, S, mask, idx, (cudaStream_t)stream);
 }
 
+veda_status veda_quantize_fp8(const float* W, int64_t H, int64_t d, uint8_t* W8, float* scale,
+                              veda_stream_t stream) {
+    if (H < 1 || d < 1 || H > (1 << 20) || d > 4096)
+        return fail(VEDA_ERR_INVALID_ARG, "fp8 weights: 1 <= H <= 2^20, 1 <= d <= 4096");
+    veda_status st;
+    if ((st = check_ptr(W, "W")) || (st = check_ptr(W8, "W8")) || (st = check_ptr(scale, "scale")))
+        return st;
+    return launch_quantize_e4m3(W, (int)H, (long long)d * d, W8, scale, (cudaStream_t)stream);
+}
+
+veda_status veda_dequantize_fp8(const uint8_t* W8, const float* scale, int64_t H, int64_t d,
+                                float* W, veda_stream_t stream) {
+    if (H < 1 || d < 1 || H > (1 << 20) || d > 4096)
+        return fail(VEDA_ERR_INVALID_ARG, "fp8 weights: 1 <= H <= 2^20, 1 <= d <= 4096");
+    veda_status st;
+    if ((st = check_ptr(W8, "W8")) || (st = check_ptr(scale, "scale")) || (st = check_ptr(W, "W")))
+        return st;
+    return launch_dequantize_e4m3(W8, scale, (int)H, (long long)d * d, W, (cudaStream_t)stream);
+}
+
 veda_status veda_mask_fused(const veda_problem* p, const float* statsQ, const float* statsK,
                             const float* Wq, const float* Wk, uint8_t* mask, int32_t* idx,
                             void* ws, veda_stream_t stream) {
