@@ -314,7 +314,8 @@ def run_veda(args, w, world, rank, local):
         dense_ms = e0.elapsed_time(e1)
 
     # end to end through the public call with host buffers (pinned), every step:
-    # H2D of Q, K, V, Wq, Wk; veda_forward; D2H of O.
+    # veda_forward_host copies Q, K, V, Wq, Wk in, runs the layer and copies O
+    # out, pipelined over chunks of heads (copies overlap the kernels).
     e2e = None
     if not args.no_e2e:
         hostQ = t["Q"].cpu().pin_memory()
@@ -328,13 +329,8 @@ def run_veda(args, w, world, rank, local):
         fws = vb.alloc_workspace(prob, dev)
 
         def e2e_step():
-            dQ.copy_(hostQ, non_blocking=True)
-            dK.copy_(hostK, non_blocking=True)
-            dV.copy_(hostV, non_blocking=True)
-            dWq.copy_(hostWq, non_blocking=True)
-            dWk.copy_(hostWk, non_blocking=True)
-            vb.veda_forward(prob, dQ, dK, dV, dWq, dWk, O, None, None, None, fws)
-            hostO.copy_(O, non_blocking=True)
+            vb.veda_forward_host(prob, hostQ, hostK, hostV, hostWq, hostWk, hostO, None, dQ, dK,
+                                 dV, dWq, dWk, O, None, fws, 0)
 
         for _ in range(min(2, args.warmup)):
             e2e_step()
@@ -404,6 +400,72 @@ def run_veda(args, w, world, rank, local):
 
 
 # ---------------------------------------------------------------- next rows
+def run_sweep(args):
+    """The sweep: H=24, d=128, 48x80 latent plane, T frames, sparsity levels
+    (one JSON line per point: layer time, effective TFLOP/s, and the speedup of
+    the attention and of the layer over the dense schedule at the same T)."""
+    import tile_sparse_attention_b200 as vb
+    vb.load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = _peaks()
+
+    def timed(fn, reps, warm=2):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps
+
+    for T in workloads.SWEEP_T:
+        w0 = workloads.sweep(T, workloads.SWEEP_SPARSITY[0])
+        t = workloads.generate(w0, device=dev)
+        B, H, N, d, nT = w0.B, w0.H, w0.N, w0.d, w0.nT
+        statsQ = torch.empty((B, H, nT, 3, d), dtype=torch.float32, device=dev)
+        statsK = torch.empty_like(statsQ)
+        S = torch.empty((B, H, nT, nT), dtype=torch.float32, device=dev)
+        O = torch.empty_like(t["Q"])
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        dense_ms = None
+        for sp in workloads.SWEEP_SPARSITY:
+            w = workloads.sweep(T, sp)
+            prob = vb.Problem.from_workload(w)
+            ws = vb.alloc_workspace(prob, dev)
+            idx = torch.empty((B, H, nT, w.k), dtype=torch.int32, device=dev)
+            if dense_ms is None:
+                dense_ms = timed(lambda: vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], None, O,
+                                                             lse, ws), reps=2, warm=1)
+
+            def layer():
+                vb.veda_tripool(prob, t["Q"], t["K"], statsQ, statsK)
+                vb.veda_tile_score(prob, statsQ, statsK, t["Wq"], t["Wk"], S, ws)
+                vb.veda_topk_mask(prob, S, None, idx)
+                vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O, lse, ws)
+            reps = 3 if w.k * nT <= 400_000 else 2
+            ms = timed(layer, reps)
+            attn_ms = timed(lambda: vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O, lse,
+                                                        ws), reps)
+            print(json.dumps({"row": "sweep", "workload": w.name, "T": T, "tokens": N, "tiles": nT,
+                              "sparsity_pct": sp, "k": w.k, "ms_per_layer": ms, "attn_ms": attn_ms,
+                              "TFLOP_s": w.sparse_flops() / (ms * 1e-3) / 1e12,
+                              "attn_TFLOP_s": w.sparse_flops() / (attn_ms * 1e-3) / 1e12,
+                              "attn_frac_bf16_burst": w.sparse_flops() / (attn_ms * 1e-3) / 1e12
+                              / peaks["bf16"],
+                              "dense_attn_ms": dense_ms, "speedup_attention": dense_ms / attn_ms,
+                              "speedup_layer": dense_ms / ms, "status": vb.veda_get_status(ws)}),
+                  flush=True)
+            del ws, idx
+        del t, statsQ, statsK, S, O, lse
+        torch.cuda.empty_cache()
+    return 0
+
+
 def run_rows(args, w, rows):
     """Times the training-side rows on `w` (one JSON line per row)."""
     import tile_sparse_attention_b200 as vb
@@ -529,6 +591,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the sweep points (T x sparsity) instead")
     ap.add_argument("--rows", default="",
                     help="comma list of f1,f2,f3,f4: time the next rows instead")
     args = ap.parse_args()
@@ -539,6 +603,8 @@ def main():
         w = workloads.sweep(int(T), int(s))
     else:
         w = workloads.CONFIGS[args.workload]()
+    if args.sweep:
+        return run_sweep(args)
     if args.rows:
         return run_rows(args, w, set(args.rows.split(",")))
     world, rank, local = _dist_init()

@@ -194,6 +194,30 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
                          veda_stream_t stream);
 
 /*
+ * The whole layer from HOST memory, pipelined over chunks of heads (every step
+ * of the layer is independent per batch entry and head): chunk g+1 is copied
+ * in on an internal copy stream while chunk g runs veda_forward's kernels on
+ * `stream`, and chunk g-1's O is copied out on a second copy stream.  Results
+ * equal one veda_forward call on the whole problem.
+ *   hQ, hK, hV: host bf16 [B, H, N, d]      hWq, hWk: host fp32 [H, d, d]
+ *   hO        : host bf16 [B, H, N, d]      hlse: host fp32 [B, H, N] or NULL
+ *   dQ, dK, dV, dO: device bf16 [B, H, N, d] staging (owned by the caller)
+ *   dWq, dWk  : device fp32 [H, d, d] staging
+ *   dlse      : device fp32 [B, H, N] staging, needed when hlse is not NULL
+ *   ws        : at least veda_workspace_size() bytes
+ *   head_chunk: heads per chunk, 1..H (0 picks H/8, at least 1)
+ * Host buffers should be page-locked (cudaHostAlloc / pinned) for the copies
+ * to overlap the kernels; with pageable memory the copies are synchronous.
+ * When `stream` completes, hO (and hlse) hold the results.  The status word in
+ * ws covers every chunk (veda_get_status).
+ */
+veda_status veda_forward_host(const veda_problem* p, const uint16_t* hQ, const uint16_t* hK,
+                              const uint16_t* hV, const float* hWq, const float* hWk,
+                              uint16_t* hO, float* hlse, uint16_t* dQ, uint16_t* dK, uint16_t* dV,
+                              float* dWq, float* dWk, uint16_t* dO, float* dlse, void* ws,
+                              int32_t head_chunk, veda_stream_t stream);
+
+/*
  * Head-aware tile search (project page, "Head-Aware Tile Search"; "Principle
  * 02 Head-Conditioned Tile Geometry"): for each head, the candidate tiling pi
  * (p_t, p_h, p_w with the same product) that minimises

@@ -65,6 +65,9 @@ def load_library(path: str = LIB_PATH):
     lib.veda_tile_score.restype = st
     lib.veda_topk_mask.argtypes = [ctypes.POINTER(veda_problem), _P, _P, _P, _P]
     lib.veda_topk_mask.restype = st
+    lib.veda_forward_host.argtypes = ([ctypes.POINTER(veda_problem)] + [_P] * 15
+                                      + [ctypes.c_int32, _P])
+    lib.veda_forward_host.restype = st
     lib.veda_quantize_fp8.argtypes = [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P]
     lib.veda_quantize_fp8.restype = st
     lib.veda_dequantize_fp8.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int64, _P, _P]
@@ -178,6 +181,30 @@ def veda_topk_mask(problem: Problem, S, mask, idx, stream=None) -> None:
     _expect(idx, torch.int32, "idx")
     _check(load_library().veda_topk_mask(ctypes.byref(problem.c), _ptr(S), _ptr(mask), _ptr(idx),
                                          _stream(stream)))
+
+
+def _host_ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("host buffers must live in host memory")
+    if not t.is_contiguous():
+        raise ValueError("host buffers must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def veda_forward_host(problem: Problem, hQ, hK, hV, hWq, hWk, hO, hlse, dQ, dK, dV, dWq, dWk, dO,
+                      dlse, ws, head_chunk: int = 0, stream=None) -> None:
+    """The layer from host buffers (pinned for overlap), pipelined over head chunks."""
+    for t, n in ((hQ, "hQ"), (hK, "hK"), (hV, "hV"), (hO, "hO"), (dQ, "dQ"), (dK, "dK"),
+                 (dV, "dV"), (dO, "dO")):
+        _expect(t, torch.bfloat16, n)
+    for t, n in ((hWq, "hWq"), (hWk, "hWk"), (dWq, "dWq"), (dWk, "dWk")):
+        _expect(t, torch.float32, n)
+    _check(load_library().veda_forward_host(
+        ctypes.byref(problem.c), _host_ptr(hQ), _host_ptr(hK), _host_ptr(hV), _host_ptr(hWq),
+        _host_ptr(hWk), _host_ptr(hO), _host_ptr(hlse), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dWq),
+        _ptr(dWk), _ptr(dO), _ptr(dlse), _ptr(ws), int(head_chunk), _stream(stream)))
 
 
 def veda_quantize_fp8(W, W8, scale, stream=None) -> None:

@@ -110,6 +110,13 @@ veda_status forward_impl(const Problem& pr, const uint16_t* Q, const uint16_t* K
                          float* lse, int32_t* idx_out, uint8_t* mask_out, void* ws,
                          cudaStream_t s);
 
+// veda_forward on host buffers, pipelined over chunks of head_chunk heads.
+veda_status forward_host_impl(const veda_problem* p, const Problem& pr, const uint16_t* hQ,
+                              const uint16_t* hK, const uint16_t* hV, const float* hWq,
+                              const float* hWk, uint16_t* hO, float* hlse, uint16_t* dQ,
+                              uint16_t* dK, uint16_t* dV, float* dWq, float* dWk, uint16_t* dO,
+                              float* dlse, void* ws, int head_chunk, cudaStream_t s);
+
 // Workspace layout of veda_forward (byte offsets, 256-aligned).
 struct WorkspaceLayout {
     size_t status, statsQ, statsK, qt, kt, S, idx, total;

@@ -287,6 +287,28 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
     return forward_impl(pr, Q, K, V, Wq, Wk, O, lse, idx_out, mask_out, ws, s);
 }
 
+veda_status veda_forward_host(const veda_problem* p, const uint16_t* hQ, const uint16_t* hK,
+                              const uint16_t* hV, const float* hWq, const float* hWk,
+                              uint16_t* hO, float* hlse, uint16_t* dQ, uint16_t* dK, uint16_t* dV,
+                              float* dWq, float* dWk, uint16_t* dO, float* dlse, void* ws,
+                              int32_t head_chunk, veda_stream_t stream) {
+    Problem pr;
+    veda_status st;
+    if ((st = make_problem(p, true, &pr)) != VEDA_OK) return st;
+    if (hQ == nullptr || hK == nullptr || hV == nullptr || hWq == nullptr || hWk == nullptr ||
+        hO == nullptr)
+        return fail(VEDA_ERR_INVALID_ARG, "host buffers must be non-NULL");
+    if ((st = check_ptr(dQ, "dQ")) || (st = check_ptr(dK, "dK")) || (st = check_ptr(dV, "dV")) ||
+        (st = check_ptr(dWq, "dWq")) || (st = check_ptr(dWk, "dWk")) || (st = check_ptr(dO, "dO")) ||
+        (st = check_ptr(dlse, "dlse", hlse == nullptr)) || (st = check_ptr(ws, "ws")))
+        return st;
+    if (head_chunk < 0 || head_chunk > pr.H)
+        return fail(VEDA_ERR_INVALID_ARG, "head_chunk must be in 0..H");
+    if (head_chunk == 0) head_chunk = pr.H / 8 > 0 ? pr.H / 8 : 1;
+    return forward_host_impl(p, pr, hQ, hK, hV, hWq, hWk, hO, hlse, dQ, dK, dV, dWq, dWk, dO,
+                             hlse ? dlse : nullptr, ws, head_chunk, (cudaStream_t)stream);
+}
+
 veda_status veda_tile_search(const veda_problem* p, const int32_t* candidates, int32_t ncand,
                              const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                              const float* Wq, const float* Wk, uint16_t* O_dense,
