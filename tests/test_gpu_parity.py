@@ -223,20 +223,28 @@ def test_forward_480p(vb, oracle):
 
 
 def test_forward_720p(vb, oracle):
+    """Mask prep of every head in full; attention on 16 seeded query tiles of every
+    head, tiles 0 and nT-1 included."""
     w = workloads.p720()
-    _forward_parity(vb, oracle, w, [0, 13, 26, 39], 6)
+    _forward_parity(vb, oracle, w, list(range(w.H)), 16)
 
 
 def test_forward_long_video(vb, oracle):
-    """245,760 tokens, 1,920 tiles, k = 96: full-size launch, sampled heads and tiles."""
+    """245,760 tokens, 1,920 tiles, k = 96, the launch the benchmark times: mask
+    prep of every head in full, attention on 16 query tiles of every head."""
     w = workloads.long_video()
-    _forward_parity(vb, oracle, w, [0, 31], 4)
+    _forward_parity(vb, oracle, w, list(range(w.H)), 16)
 
 
-@pytest.mark.parametrize("T,s", [(4, 0), (4, 98), (8, 50), (20, 80), (32, 90), (64, 95)])
+@pytest.mark.parametrize("T", workloads.SWEEP_T)
+@pytest.mark.parametrize("s", workloads.SWEEP_SPARSITY)
 def test_forward_sweep_points(vb, oracle, T, s):
+    """Every sweep point: mask prep of every head in full; attention on 16 query
+    tiles of every head (fewer where k is large: the oracle's work per tile
+    grows with k), tiles 0 and nT-1 always included."""
     w = workloads.sweep(T, s)
-    _forward_parity(vb, oracle, w, [0, 23], 3)
+    per_head = max(2, min(16, (16 * 96) // w.k))
+    _forward_parity(vb, oracle, w, list(range(w.H)), per_head)
 
 
 def test_sweep_k_all_matches_dense_path(vb):
