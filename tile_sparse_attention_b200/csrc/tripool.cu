@@ -10,8 +10,8 @@
 // p_t*p_h runs of p_w contiguous tokens (a token row is d bf16 = 128 or 256
 // bytes).  Thread t owns channel group (t % G) (8 channels = 16 bytes) and
 // token lane (t / G); it walks its tokens with all loads issued up front, then
-// the token lanes are reduced through shared memory.  Output rows (avg, max,
-// min) are written as coalesced fp32.
+// the token lanes are reduced by warp shuffles and across the four warps through
+// shared memory.  Output rows (avg, max, min) are written as coalesced fp32.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(128) tripool_kernel(const __grid_constant__ Tr
     constexpr int G = D / 8;            // 16-byte channel groups per token row
     constexpr int LANES = 128 / G;      // token lanes
     constexpr int PER = BT / LANES;     // tokens per thread
-    __shared__ float red[3][LANES][D];
+    __shared__ float red[3][4][8][G];  // [statistic][warp][channel in group][group]
 
     const int j = blockIdx.x;           // tile
     const int bh = blockIdx.y;          // b*H + h
@@ -58,13 +58,27 @@ __global__ void __launch_bounds__(128) tripool_kernel(const __grid_constant__ Tr
     const int lane_tok = threadIdx.x / G;
     const uint16_t* base = p.X[which] + (size_t)bh * p.N * D;
 
+    // Row r = lane_tok + i*LANES of the tile is token (lt, lh, lw) of the box
+    // in raster order; the position is computed once and then advanced by
+    // LANES rows with carries (no division per load).
+    int lw = lane_tok % pw, lh = (lane_tok / pw) % ph, lt = lane_tok / (ph * pw);
+    const int step_w = LANES % pw, step_h = (LANES / pw) % ph, step_t = LANES / (ph * pw);
     uint4 v[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-        const int r = lane_tok + i * LANES;           // row of the tile
-        const int lt = r / (ph * pw), lh = (r / pw) % ph, lw = r % pw;
         const int n = ((a * pt + lt) * p.Hs + (b * ph + lh)) * p.Ws + (c * pw + lw);
         v[i] = __ldg(reinterpret_cast<const uint4*>(base + (size_t)n * D) + g);
+        lw += step_w;
+        lh += step_h;
+        lt += step_t;
+        if (lw >= pw) {
+            lw -= pw;
+            ++lh;
+        }
+        if (lh >= ph) {
+            lh -= ph;
+            ++lt;
+        }
     }
     float sum[8], mx[8], mn[8];
 #pragma unroll
@@ -84,21 +98,36 @@ __global__ void __launch_bounds__(128) tripool_kernel(const __grid_constant__ Tr
             mn[e] = fminf(mn[e], f[e]);
         }
     }
+    // token lanes that sit in the same warp hold the same channels: combine them
+    // with shuffles, then the four warps through shared memory ([e][g] order, so
+    // the 16-byte channel groups of a warp land in distinct banks)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        red[0][lane_tok][g * 8 + e] = sum[e];
-        red[1][lane_tok][g * 8 + e] = mx[e];
-        red[2][lane_tok][g * 8 + e] = mn[e];
+    for (int off = G; off < 32; off <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            sum[e] += __shfl_xor_sync(0xffffffffu, sum[e], off);
+            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
+            mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], off));
+        }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane < G) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            red[0][warp][e][g] = sum[e];
+            red[1][warp][e][g] = mx[e];
+            red[2][warp][e][g] = mn[e];
+        }
     }
     __syncthreads();
     float* out = p.out[which] + ((size_t)bh * p.nT + j) * 3 * D;
     for (int ch = threadIdx.x; ch < D; ch += 128) {
+        const int cg = ch >> 3, ce = ch & 7;
         float s = 0.f, M = -INFINITY, m = INFINITY;
 #pragma unroll
-        for (int l = 0; l < LANES; ++l) {
-            s += red[0][l][ch];
-            M = fmaxf(M, red[1][l][ch]);
-            m = fminf(m, red[2][l][ch]);
+        for (int w = 0; w < 4; ++w) {
+            s += red[0][w][ce][cg];
+            M = fmaxf(M, red[1][w][ce][cg]);
+            m = fminf(m, red[2][w][ce][cg]);
         }
         out[ch] = s * (1.0f / BT);
         out[D + ch] = M;
