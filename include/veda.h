@@ -10,10 +10,12 @@
  *
  * Conventions shared by every call
  * --------------------------------
- * - Every pointer except `veda_problem::tile_shapes` is a caller-owned DEVICE
- *   pointer.  The library never allocates, frees or keeps a pointer after the
- *   call returns.  All work is enqueued asynchronously on `stream`; results are
- *   ready when the stream reaches that point.
+ * - Every pointer is a caller-owned DEVICE pointer, except
+ *   `veda_problem::tile_shapes` and the pointers a call names HOST (the host
+ *   buffers of veda_forward_host, the candidates of veda_tile_search).  The
+ *   library never allocates, frees or keeps a pointer after the call returns.
+ *   All work is enqueued asynchronously on `stream`; results are ready when the
+ *   stream reaches that point.
  * - Tensors are dense and row-major.  Q, K, V, O are bf16 (passed as uint16_t
  *   bit patterns) of shape [B, H, N, d] with N = T*Hs*Ws tokens in raster
  *   (t, y, x) order: token n = (t*Hs + y)*Ws + x.
@@ -133,7 +135,8 @@ veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask,
  *   W    : fp32 [H, d, d] (device)      W8: uint8 [H, d, d]      scale: fp32 [H]
  * veda_dequantize_fp8 writes the fp32 weights fp32(E4M3(W8) * scale[h]), which
  * veda_tile_score / veda_mask_fused / veda_forward take as Wq, Wk.
- * Errors: VEDA_ERR_INVALID_ARG (H < 1, d < 1 or a NULL pointer).
+ * Errors: VEDA_ERR_INVALID_ARG (H outside 1..2^20, d outside 1..4096, or a NULL
+ * pointer), VEDA_ERR_ALIGN (a pointer not 16-byte aligned).
  */
 veda_status veda_quantize_fp8(const float* W, int64_t H, int64_t d, uint8_t* W8, float* scale,
                               veda_stream_t stream);
