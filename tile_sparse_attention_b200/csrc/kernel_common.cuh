@@ -60,6 +60,14 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity, co
     return ok != 0;
 }
 
+// Order-preserving 32-bit key of a finite fp32 score: a larger score gives a
+// larger key; -0.0 and +0.0 give the same key.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    uint32_t u = __float_as_uint(v);
+    if ((u << 1) == 0) u = 0;  // -0.0 -> +0.0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Grid origin (t0, y0, x0) of tile t for tile shape (pt, ph, pw).
 __device__ __forceinline__ void tile_origin(int t, int pt, int ph, int pw, int Hs, int Ws,
                                             int& t0, int& y0, int& x0) {

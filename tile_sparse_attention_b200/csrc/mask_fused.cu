@@ -76,31 +76,6 @@ struct __align__(64) FusedParams {
     unsigned long long wait_limit_ns;
 };
 
-__device__ __forceinline__ uint32_t order_key(float v) {
-    uint32_t u = __float_as_uint(v);
-    if ((u << 1) == 0) u = 0;  // -0.0 -> +0.0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(kIdescTF32F), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_rows(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                              int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
-        : "memory");
-}
-
 // Min-heap of `n` entries of one row: entry e at heap[e * 128] (entry-major,
 // so the 128 rows' heaps interleave and equal positions hit distinct banks).
 __device__ __forceinline__ void sift_down(uint64_t* heap, int pos, int n) {
@@ -196,8 +171,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                     }
                     uint8_t* a = smem + st * kStageBytesF;
                     mbar_arrive_expect_tx(&full[st], kStageBytesF);
-                    tma_load_rows(a, &p.mapA, &full[st], kb * 32, rowA);
-                    tma_load_rows(a + kTileBytesF, &p.mapB, &full[st], kb * 32, rowB);
+                    tma_load_2d(a, &p.mapA, &full[st], kb * 32, rowA);
+                    tma_load_2d(a + kTileBytesF, &p.mapB, &full[st], kb * 32, rowB);
                     issued = g + 1;
                 }
             }
@@ -227,7 +202,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = smem_desc_sw128(a + kk * 32, 16, 1024);
                         const uint64_t bd = smem_desc_sw128(a + kTileBytesF + kk * 32, 16, 1024);
-                        mma_tf32(tbase + b * 128, ad, bd, (kb > 0 || kk > 0) ? 1u : 0u);
+                        mma_tf32_ss(tbase + b * 128, ad, bd, kIdescTF32F, (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(&empty[st]);
                 }

@@ -22,6 +22,7 @@
 // Waits are bounded (VEDA_ERR_TIMEOUT in the status word, then a bounded drain
 // of the copies and products in flight before tensor memory is freed).
 #include "internal.h"
+#include "kernel_common.cuh"
 #include "ptx.cuh"
 
 namespace veda {
@@ -46,39 +47,6 @@ struct __align__(64) ScoreParams {
     unsigned long long wait_limit_ns;
 };
 
-__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-// Bounded wait (suspending in hardware between tests); false on expiry.
-__device__ __forceinline__ bool wait_limited(uint64_t* bar, uint32_t parity,
-                                             const ScoreParams& p) {
-    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait_sleep(bar, parity, 20000)) {
-        if (global_timer_ns() - t0 > p.wait_limit_ns) {
-            atomicCAS(p.status, 0, (int)VEDA_ERR_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
-}
-
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_tc_kernel(const __grid_constant__ ScoreParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -89,6 +57,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     uint64_t* done = empty + kStages;
     uint64_t* drain = done + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int j0 = blockIdx.x * 128, i0 = blockIdx.y * 128, bh = blockIdx.z;
@@ -102,6 +71,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
         mbar_init(done, 1);
         mbar_init(drain, 1);
+        *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -121,7 +91,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         int issued = 0;
         for (int kb = 0; kb < KB; ++kb) {
             const int st = kb % kStages, n = kb / kStages;
-            if (n > 0 && !wait_limited(&empty[st], (n - 1) & 1, p)) break;
+            if (n > 0 && !wait_bar(&empty[st], (n - 1) & 1, p, abort_flag)) break;
             uint8_t* a = smem + st * kStageBytes;
             mbar_arrive_expect_tx(&full[st], kStageBytes);
             tma_load_2d(a, &p.mapA, &full[st], kb * 32, rowA);
@@ -129,13 +99,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             issued = kb + 1;
         }
         for (int st = 0; st < kStages; ++st)  // drain: the last fill of every stage
-            if (st < issued) wait_limited(&full[st], ((issued - 1 - st) / kStages) & 1, p);
+            if (st < issued) drain_bar(&full[st], ((issued - 1 - st) / kStages) & 1, p);
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------- MMA issuer
         const uint32_t base = smem_addr(smem);
         for (int kb = 0; kb < KB && ok; ++kb) {
             const int st = kb % kStages;
-            if (!wait_limited(&full[st], (kb / kStages) & 1, p)) {
+            if (!wait_bar(&full[st], (kb / kStages) & 1, p, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -151,13 +121,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
         mma_commit(done);
         mma_commit(drain);
-        wait_limited(drain, 0, p);
+        drain_bar(drain, 0, p);
     }
     __syncwarp();
 
     // -------------------------------------------------------------- epilogue
     int got = 0;
-    if (lane == 0) got = wait_limited(done, 0, p) ? 1 : 0;
+    if (lane == 0) got = wait_bar(done, 0, p, abort_flag) ? 1 : 0;
     got = __shfl_sync(0xffffffffu, got, 0);
     __syncwarp();
     if (got) {

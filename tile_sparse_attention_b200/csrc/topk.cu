@@ -15,16 +15,11 @@
 // pop-counts, the index list already sorted.  The selection is an integer
 // computation on the fp32 scores, so it is exactly reproducible.
 #include "internal.h"
+#include "kernel_common.cuh"
 
 namespace veda {
 
 namespace {
-
-__device__ __forceinline__ uint32_t order_key(float v) {
-    uint32_t u = __float_as_uint(v);
-    if ((u << 1) == 0) u = 0;  // -0.0 -> +0.0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 struct TopkParams {
     const float* S;
