@@ -5,7 +5,9 @@ first "P ready" arrival, so the tensor-core issuer's bounded wait (limit set to
 300 ms through VEDA_WAIT_LIMIT_MS) expires.  The CTA then raises its abort
 flag, the other roles leave their waits, in-flight copies and products are
 drained, tensor memory is freed and VEDA_ERR_TIMEOUT lands in the status word.
-The context stays usable: the next call computes correct results.
+The context stays usable: the next call computes correct results.  Both
+attention kernels are covered: the persistent one (short key lists) and the
+one-CTA-per-query-tile one (k above 64).
 """
 import os
 
@@ -18,13 +20,19 @@ import workloads
 
 pytestmark = pytest.mark.gpu
 
+CASES = [
+    ("persistent_k2", workloads.tiny),
+    ("per_tile_k80", lambda: workloads.custom("wb", 1, 2, 128, (8, 32, 64), [(2, 8, 8)], 80)),
+]
 
-def test_timeout_is_reported_and_context_survives(oracle):
+
+@pytest.mark.parametrize("name,make", CASES)
+def test_timeout_is_reported_and_context_survives(oracle, name, make):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import tile_sparse_attention_b200 as vb
     vb.load_library()
-    w = workloads.tiny()
+    w = make()
     t = {n: v.cuda() for n, v in workloads.generate(w, device="cpu").items()}
     prob = vb.Problem.from_workload(w)
     idx = torch.stack([torch.arange(w.k, dtype=torch.int32)] * (w.H * w.nT)).reshape(
@@ -45,7 +53,7 @@ def test_timeout_is_reported_and_context_survives(oracle):
     vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O, lse, ws)
     assert vb.veda_get_status(ws) == 0
     bits = {n: ph.to_host_bits(t[n]) for n in "QKV"}
-    units = np.array([(0, h, i) for h in range(w.H) for i in range(w.nT)], dtype=np.int64)
+    units = workloads.sample_units(w, min(w.nT, 8), seed=5)
     O_o, lse_o, toks = oracle.sparse_attention(bits["Q"], bits["K"], bits["V"], idx.cpu().numpy(),
                                                w.grid, w.tile_shapes, w.scale, units=units)
     ph.check_attention(ph.to_host_bits(O), lse.cpu().numpy(), units, O_o, lse_o, toks)

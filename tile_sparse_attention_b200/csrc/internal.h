@@ -63,6 +63,13 @@ veda_status launch_topk(const Problem& pr, const float* S, uint8_t* mask, int32_
 veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint16_t* K,
                                const uint16_t* V, const int32_t* idx, int k, uint16_t* O,
                                float* lse, int* status, cudaStream_t s);
+// The persistent-CTA kernel for short key lists (launch_sparse_attn uses it
+// for k <= kPersistentMaxK).
+constexpr int kPersistentMaxK = 64;
+veda_status launch_sparse_attn_persistent(const Problem& pr, const uint16_t* Q,
+                                          const uint16_t* K, const uint16_t* V,
+                                          const int32_t* idx, int k, uint16_t* O, float* lse,
+                                          int* status, cudaStream_t s);
 
 // TMA descriptors (tensor_maps.cu): the 5-D tile view (d, Ws, Hs, T, B*H) of a
 // [B,H,N,d] bf16 tensor with a (64, p_w, p_h, p_t, 1) box, and a 2-D row view

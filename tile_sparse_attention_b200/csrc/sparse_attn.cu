@@ -1,4 +1,6 @@
-// sparse_attn.cu -- tile-skipping flash attention for sm_100a (tcgen05 + TMEM + TMA).
+// sparse_attn.cu -- tile-skipping flash attention for sm_100a (tcgen05 + TMEM + TMA),
+// one CTA per query tile (used for k > kPersistentMaxK; shorter key lists go to
+// the persistent kernel in sparse_attn_persistent.cu).
 //
 // "Veda: Scalable Video Diffusion via Distilled Sparse Attention" (project
 // page): "Attention Structure Distillation", Execution (the tile mask is
@@ -516,6 +518,11 @@ veda_status launch_cfg(const AttnParams& prm, const Problem& pr, cudaStream_t s)
 veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint16_t* K,
                                const uint16_t* V, const int32_t* idx, int k, uint16_t* O,
                                float* lse, int* status, cudaStream_t s) {
+    // Short key lists: the per-CTA fixed cost (allocation, Q load, pipeline fill,
+    // epilogue) dominates, and the persistent kernel that carries its pipeline
+    // across query tiles is faster; long ones: this kernel's steady state is.
+    if (k <= kPersistentMaxK)
+        return launch_sparse_attn_persistent(pr, Q, K, V, idx, k, O, lse, status, s);
     AttnParams prm;
     memset(&prm, 0, sizeof(prm));
     for (int sh = 0; sh < pr.nshapes; ++sh) {
