@@ -78,6 +78,36 @@ def test_topk_bit_exact_on_given_scores(vb, oracle):
         np.testing.assert_array_equal(mask.cpu().numpy(), m_o)
 
 
+def test_topk_bit_exact_on_extreme_rows(vb, oracle):
+    """Rows that defeat value bucketing: one huge outlier (every other score in one
+    bucket), constant rows, a range beyond fp32 (max - min overflows), sub-normal
+    spacing, coarse quantisation (hundreds of equal scores at the threshold), and
+    k = nT.  The selection must still equal the oracle's exactly."""
+    rng = np.random.default_rng(11)
+    for nT, k in ((1920, 96), (600, 30), (37, 5), (300, 300), (4097, 200)):
+        H = 8
+        w = workloads.custom("topk_x", 1, H, 64, (1, 1, 64 * nT), [(1, 1, 64)], k)
+        S = rng.standard_normal((1, H, nT, nT)).astype(np.float32)
+        S[0, 0, :, nT // 3] = 1e30                                   # outlier column
+        S[0, 1] = 2.5                                                # constant rows
+        S[0, 2, :, 0] = 3e38
+        S[0, 2, :, -1] = -3e38                                       # max - min = inf
+        S[0, 3] = (rng.integers(0, 6, (nT, nT)) * 1e-45).astype(np.float32)  # sub-normals
+        S[0, 4] = np.round(S[0, 4] * 2) / 2                          # many equal scores
+        S[0, 5] = np.abs(S[0, 5]) * 1e-3 + 7.0                       # narrow range, far from 0
+        S[0, 6, :, ::2] = -0.0
+        S[0, 6, :, 1::2] = 0.0                                       # only signed zeros
+        S[0, 7] = -np.abs(S[0, 7])                                   # all negative
+        prob = vb.Problem.from_workload(w)
+        mask = torch.empty((1, H, nT, nT), dtype=torch.uint8, device="cuda")
+        idx = torch.empty((1, H, nT, k), dtype=torch.int32, device="cuda")
+        vb.veda_topk_mask(prob, torch.from_numpy(S).cuda(), mask, idx)
+        rows = np.arange(nT) if nT <= 2048 else np.unique(rng.integers(0, nT, 64))
+        m_o, i_o = oracle.topk(S[:, :, rows].astype(np.float64), k)
+        np.testing.assert_array_equal(idx[:, :, rows].cpu().numpy(), i_o)
+        np.testing.assert_array_equal(mask[:, :, rows].cpu().numpy(), m_o)
+
+
 # ------------------------------------------------------------------ attention
 def _attn_case(vb, oracle, w, t, idx_np, units, dense=False):
     prob = vb.Problem.from_workload(w)

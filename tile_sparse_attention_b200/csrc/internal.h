@@ -33,6 +33,8 @@ veda_status make_problem(const veda_problem* p, bool need_k, Problem* out);
 veda_status check_ptr(const void* ptr, const char* name, bool nullable = false);
 
 veda_status cuda_check(cudaError_t err, const char* what);
+// SMs of the current device (1 if the query fails).
+int sm_count();
 
 // Launchers (defined next to their kernels).  Each returns VEDA_OK or an
 // error after checking the launch.

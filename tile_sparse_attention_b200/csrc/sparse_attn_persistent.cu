@@ -553,14 +553,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
-        return 1;
-    return n;
-}
-
 template <int D, int BT, int NS>
 veda_status launch_cfg(const AttnParams& prm, const Problem& pr, cudaStream_t s) {
     using C = Cfg<D, BT, NS>;

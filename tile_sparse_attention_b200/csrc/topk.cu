@@ -6,20 +6,34 @@
 // query tile produces the tile mask handed to the tile-skipping kernel.  Ties
 // go to the lower tile index; -0.0 and +0.0 tie.
 //
-// One warp per row.  Scores become order-preserving 32-bit keys (larger score
-// -> larger key), held in shared memory.  An exact radix select (8 bits per
-// pass, most significant first, over the bits in which the row's keys differ)
-// finds the k-th largest key K* and how many keys equal to K* are kept (the
-// lowest-index ones).  A final pass in
-// ascending index order emits the mask and, through warp ballots and prefix
-// pop-counts, the index list already sorted.  The selection is an integer
-// computation on the fp32 scores, so it is exactly reproducible.
+// One warp per row.  The row is read with 16-byte loads (up to sixteen in flight
+// per lane) into shared memory.  The selection is exact and integer-valued:
+//   1. Bucketing: every score goes to one of 256 buckets spread linearly over
+//      [row min, row max].  The bucket index is computed with correctly
+//      rounded fp32 operations from the score alone, so it is a
+//      non-decreasing function of the score (equal scores, -0.0 and +0.0
+//      included, share a bucket).  A histogram gives the bucket b* holding
+//      the k-th largest score and the count of scores in higher buckets, all
+//      of which are selected.
+//   2. Within b* (a handful of scores for smooth score distributions), the
+//      exact threshold key K* (order-preserving 32-bit keys, larger score ->
+//      larger key) and how many keys equal to K* are kept: pairwise ranks for
+//      at most 32 candidates, else a radix select (8 bits per pass, most
+//      significant varying bit first) over the candidates.
+//   3. One pass in ascending index order emits the mask (four bytes per lane
+//      store) and, through warp ballots and prefix pop-counts, the index list
+//      already sorted; of the keys equal to K*, the lowest-index ones are kept.
+#include <cfloat>
+
 #include "internal.h"
 #include "kernel_common.cuh"
 
 namespace veda {
 
 namespace {
+
+constexpr int kBins = 256;     // buckets of the first pass and radix digits
+constexpr int kCandCap = 256;  // candidate keys kept in shared memory per row
 
 struct TopkParams {
     const float* S;
@@ -29,103 +43,315 @@ struct TopkParams {
     int nT, k;
 };
 
-template <int WARPS>
-__global__ void __launch_bounds__(WARPS * 32) topk_kernel(const __grid_constant__ TopkParams p) {
-    extern __shared__ __align__(16) uint32_t smem_u[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long row = (long long)blockIdx.x * WARPS + warp;
-    if (row >= p.rows) return;
-    const int nT = p.nT;
-    const int nT4 = (nT + 3) & ~3;
-    uint32_t* keys = smem_u + (size_t)warp * (nT4 + 256);
-    uint32_t* hist = keys + nT4;
-    const float* srow = p.S + row * nT;
+// Shared-memory words of one warp: the row (rounded up to groups of four),
+// the histogram, the candidate list and its counter (padded to 16 bytes).
+__host__ __device__ inline size_t topk_warp_words(int nT) {
+    return (size_t)4 * ((nT + 3) >> 2) + kBins + kCandCap + 4;
+}
 
-    for (int j = lane; j < nT; j += 32) keys[j] = order_key(__ldg(srow + j));
+// Bucket of score x among kBins linear buckets over [mn, mn + kBins / inv];
+// inv >= 0 and finite, x >= mn, so t is finite and >= 0 and the result is
+// non-decreasing in x.
+__device__ __forceinline__ int bucket_of(float x, float mn, float inv) {
+    const float t = __fmul_rn(__fsub_rn(x, mn), inv);
+    return t < (float)(kBins - 1) ? (int)t : kBins - 1;
+}
 
-    // Bits above the highest bit in which the row's keys differ are common to
-    // all keys: the radix passes start below them, so the first histogram is
-    // spread out instead of piling every key into one bin.
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int j = lane; j < nT; j += 32) {
-        kmin = min(kmin, keys[j]);
-        kmax = max(kmax, keys[j]);
+// The bin holding the kr-th largest element of a kBins-bin histogram (bins in
+// ascending value order, so the scan runs from the top bin down); `above`
+// receives the number of elements in higher bins.  kr must not exceed the
+// histogram's total.
+__device__ __forceinline__ uint32_t select_bin(const uint32_t* hist, int kr, int lane,
+                                               uint32_t& above) {
+    // lane l owns bins 255-8l ... 248-8l (descending)
+    uint32_t cnt[8];
+    uint32_t local = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        cnt[e] = hist[kBins - 1 - 8 * lane - e];
+        local += cnt[e];
     }
+    uint32_t incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, incl >= (uint32_t)kr);
+    const int src = __ffs(hit) - 1;
+    uint32_t bin = 0, ab = 0;
+    if (lane == src) {
+        uint32_t run = incl - local;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (run + cnt[e] >= (uint32_t)kr) {
+                bin = kBins - 1 - 8 * lane - e;
+                ab = run;
+                break;
+            }
+            run += cnt[e];
+        }
+    }
+    above = __shfl_sync(0xffffffffu, ab, src);
+    return __shfl_sync(0xffffffffu, bin, src);
+}
+
+// Exact radix select of the kr-th largest key among the candidates.  each(f)
+// calls f(key) for every candidate key held by this lane (a shared-memory list
+// or registers).  Returns that key; kr becomes the number of candidates equal
+// to it that are kept (ranked among equal keys).
+template <class Each>
+__device__ uint32_t radix_select(const Each& each, int& kr, uint32_t* hist, int lane) {
+    // Bits above the highest bit in which the candidates differ are common to
+    // all of them: the passes start below them.
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    each([&](uint32_t key) {
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+    });
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
         kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
         kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
     }
     const int top = 32 - __clz(kmin ^ kmax);  // number of bits that vary (0..32)
-    uint32_t prefix = kmin & (top == 32 ? 0u : ~((1u << top) - 1u));
     uint32_t pmask = top == 32 ? 0u : ~((1u << top) - 1u);
-    int kr = p.k;  // rank of the wanted key among the candidates, from the top
+    uint32_t prefix = kmin & pmask;
 #pragma unroll 1
     for (int hi = top; hi > 0; hi -= 8) {
         const int shift = hi >= 8 ? hi - 8 : 0;
-        const uint32_t dmask = (hi >= 8 ? 255u : (1u << hi) - 1u);
-        for (int b = lane; b < 256; b += 32) hist[b] = 0;
+        const uint32_t dmask = hi >= 8 ? 255u : (1u << hi) - 1u;
+        for (int b = lane; b < kBins; b += 32) hist[b] = 0;
         __syncwarp();
-        for (int j = lane; j < nT; j += 32) {
-            const uint32_t key = keys[j];
+        each([&](uint32_t key) {
             if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
-        }
+        });
         __syncwarp();
-        // lane l owns bins 255-8l ... 248-8l (descending digit order)
-        uint32_t cnt[8];
-        uint32_t local = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            cnt[e] = hist[255 - 8 * lane - e];
-            local += cnt[e];
-        }
-        uint32_t incl = local;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
-        }
-        const uint32_t hit = __ballot_sync(0xffffffffu, incl >= (uint32_t)kr);
-        const int src = __ffs(hit) - 1;  // kr <= candidates, so some lane hits
-        uint32_t digit = 0, above = 0;
-        if (lane == src) {
-            uint32_t run = incl - local;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                if (run + cnt[e] >= (uint32_t)kr) {
-                    digit = 255 - 8 * lane - e;
-                    above = run;
-                    break;
-                }
-                run += cnt[e];
-            }
-        }
-        digit = __shfl_sync(0xffffffffu, digit, src);
-        above = __shfl_sync(0xffffffffu, above, src);
+        uint32_t above;
+        const uint32_t digit = select_bin(hist, kr, lane, above);
         kr -= (int)above;
         prefix |= digit << shift;
         pmask |= dmask << shift;
         __syncwarp();
     }
-    const uint32_t thr = prefix;  // k-th largest key; keep kr of the keys equal to it
+    return prefix;
+}
 
+// Threshold among the c candidate keys of cand[] (c >= kr >= 1): pairwise
+// ranks for at most 32 (the lanes holding the kr-th largest key see fewer than
+// kr larger keys and at least kr larger-or-equal ones), else a radix select.
+// Returns the key; kr becomes the number of keys equal to it that are kept.
+__device__ __forceinline__ uint32_t candidate_threshold(const uint32_t* cand, int c, int& kr,
+                                                       uint32_t* hist, int lane) {
+    const unsigned full = 0xffffffffu;
+    if (c <= 32) {
+        const uint32_t mine = lane < c ? cand[lane] : 0u;
+        int gt = 0, eq = 0;
+        for (int m = 0; m < c; ++m) {
+            const uint32_t o = __shfl_sync(full, mine, m);
+            gt += o > mine ? 1 : 0;
+            eq += o == mine ? 1 : 0;
+        }
+        const bool hit = lane < c && gt < kr && gt + eq >= kr;
+        const int src = __ffs(__ballot_sync(full, hit)) - 1;
+        kr -= __shfl_sync(full, gt, src);
+        return __shfl_sync(full, mine, src);
+    }
+    return radix_select(
+        [&](auto&& f) {
+            for (int j = lane; j < c; j += 32) f(cand[j]);
+        },
+        kr, hist, lane);
+}
+
+// Score of an order key (inverse of order_key; the key of -0.0 maps to +0.0).
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+}
+
+// LOADS: 16-byte loads in flight per lane (16 for long rows; 8 keeps the
+// register count, and so the warps per SM, up for rows of up to 1024 scores).
+template <int WARPS, int LOADS>
+__global__ void __launch_bounds__(WARPS * 32) topk_kernel(const __grid_constant__ TopkParams p) {
+    extern __shared__ __align__(16) uint32_t smem_u[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * WARPS + warp;
+    if (row >= p.rows) return;
+    const int nT = p.nT;
+    const int nG = (nT + 3) >> 2;  // groups of four scores
+    uint32_t* base = smem_u + (size_t)warp * topk_warp_words(nT);
+    float* vals = reinterpret_cast<float*>(base);
+    float4* v4 = reinterpret_cast<float4*>(base);
+    uint32_t* hist = base + 4 * nG;
+    uint32_t* cand = hist + kBins;
+    uint32_t* ncand = cand + kCandCap;
+    const float* srow = p.S + row * nT;
+    const unsigned full = 0xffffffffu;
+
+    // ---- 1. the row into shared memory, with its min and max
+    float mn = INFINITY, mx = -INFINITY;
+    if ((nT & 3) == 0) {  // rows start on 16-byte boundaries (S is 16-byte aligned)
+        const float4* s4 = reinterpret_cast<const float4*>(srow);
+        for (int g = lane; g < nG; g += 32 * LOADS) {
+            float4 t[LOADS];
+#pragma unroll
+            for (int u = 0; u < LOADS; ++u)
+                if (g + 32 * u < nG) t[u] = __ldcs(s4 + g + 32 * u);
+#pragma unroll
+            for (int u = 0; u < LOADS; ++u)
+                if (g + 32 * u < nG) {
+                    v4[g + 32 * u] = t[u];
+                    mn = fminf(mn, fminf(fminf(t[u].x, t[u].y), fminf(t[u].z, t[u].w)));
+                    mx = fmaxf(mx, fmaxf(fmaxf(t[u].x, t[u].y), fmaxf(t[u].z, t[u].w)));
+                }
+        }
+    } else {
+        for (int j = lane; j < nT; j += 32 * 8) {
+            float t[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (j + 32 * u < nT) t[u] = __ldcs(srow + j + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (j + 32 * u < nT) {
+                    vals[j + 32 * u] = t[u];
+                    mn = fminf(mn, t[u]);
+                    mx = fmaxf(mx, t[u]);
+                }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(full, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(full, mx, off));
+    }
+    // kBins buckets over [mn, mx]; a zero or non-finite range puts every score
+    // in bucket 0 (still exact: the candidates are then the whole row)
+    const float range = __fsub_rn(mx, mn);
+    const float inv = (range > 0.f && range <= FLT_MAX) ? fminf((float)kBins / range, FLT_MAX) : 0.f;
+    __syncwarp();
+
+    // ---- 2. bucket histogram and the bucket of the k-th largest score
+    for (int b = lane; b < kBins; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int g = lane; g < nG; g += 32) {
+        const float4 x = v4[g];
+        const int j = 4 * g;
+        atomicAdd(&hist[bucket_of(x.x, mn, inv)], 1u);
+        if (j + 1 < nT) atomicAdd(&hist[bucket_of(x.y, mn, inv)], 1u);
+        if (j + 2 < nT) atomicAdd(&hist[bucket_of(x.z, mn, inv)], 1u);
+        if (j + 3 < nT) atomicAdd(&hist[bucket_of(x.w, mn, inv)], 1u);
+    }
+    __syncwarp();
+    uint32_t above;
+    const int bstar = (int)select_bin(hist, p.k, lane, above);
+    int kr = p.k - (int)above;  // rank of the k-th largest score within bucket b*
+    __syncwarp();
+
+    // ---- 3. the keys of bucket b* (in any order), and the exact threshold among them
+    if (lane == 0) *ncand = 0;
+    __syncwarp();
+    for (int g = lane; g < nG; g += 32) {
+        const float4 x = v4[g];
+        const float xe[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (4 * g + e < nT && bucket_of(xe[e], mn, inv) == bstar) {
+                const uint32_t pos = atomicAdd(ncand, 1u);
+                if (pos < (uint32_t)kCandCap) cand[pos] = order_key(xe[e]);
+            }
+    }
+    __syncwarp();
+    const int c = (int)*ncand;  // candidates (warp-uniform)
+    uint32_t thr;
+    if (c <= kCandCap) {
+        thr = candidate_threshold(cand, c, kr, hist, lane);
+    } else {
+        thr = radix_select(
+            [&](auto&& f) {
+                for (int j = lane; j < nT; j += 32) {
+                    const float x = vals[j];
+                    if (bucket_of(x, mn, inv) == bstar) f(order_key(x));
+                }
+            },
+            kr, hist, lane);
+    }
+
+    // scores above and equal to the threshold, compared as floats (order keys
+    // compare like the scores, with -0.0 equal to +0.0)
+    const float tv = key_value(thr);
+
+    // ---- 4. mask and ascending index list; keep the kr lowest-index scores equal to tv
     const unsigned lt_mask = (1u << lane) - 1u;
     int eq_seen = 0, sel_seen = 0;
     int32_t* irow = p.idx + row * p.k;
     uint8_t* mrow = p.mask ? p.mask + row * nT : nullptr;
-    for (int j0 = 0; j0 < nT; j0 += 32) {
-        const int j = j0 + lane;
-        const uint32_t key = j < nT ? keys[j] : 0u;
-        const bool eq = (j < nT) && key == thr;
-        const unsigned eq_b = __ballot_sync(0xffffffffu, eq);
-        const int eq_rank = eq_seen + __popc(eq_b & lt_mask);
-        const bool sel = (j < nT) && (key > thr || (eq && eq_rank < kr));
-        const unsigned sel_b = __ballot_sync(0xffffffffu, sel);
-        if (sel) irow[sel_seen + __popc(sel_b & lt_mask)] = j;
-        if (mrow && j < nT) mrow[j] = sel ? 1 : 0;
-        eq_seen += __popc(eq_b);
-        sel_seen += __popc(sel_b);
+    for (int g0 = 0; g0 < nG; g0 += 32) {
+        const int g = g0 + lane;
+        const bool gv = g < nG;
+        const float4 x = gv ? v4[g] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float xe[4] = {x.x, x.y, x.z, x.w};
+        bool eq[4], sel[4];
+        int neq = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const bool valid = gv && 4 * g + e < nT;
+            eq[e] = valid && xe[e] == tv;
+            sel[e] = valid && xe[e] > tv;
+            neq += eq[e] ? 1 : 0;
+        }
+        if (__any_sync(full, neq > 0)) {
+            int r = eq_seen, tot = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const unsigned b = __ballot_sync(full, eq[e]);
+                r += __popc(b & lt_mask);
+                tot += __popc(b);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (eq[e] && r < kr) sel[e] = true;
+                r += eq[e] ? 1 : 0;
+            }
+            eq_seen += tot;
+        }
+        int pos = sel_seen, tot = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const unsigned b = __ballot_sync(full, sel[e]);
+            pos += __popc(b & lt_mask);
+            tot += __popc(b);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (sel[e]) {
+                if (pos < p.k) irow[pos] = 4 * g + e;  // exactly k are selected
+                ++pos;
+            }
+        sel_seen += tot;
+        if (mrow != nullptr) {
+            if ((nT & 3) == 0) {
+                if (gv)
+                    reinterpret_cast<uchar4*>(mrow)[g] =
+                        make_uchar4(sel[0] ? 1 : 0, sel[1] ? 1 : 0, sel[2] ? 1 : 0, sel[3] ? 1 : 0);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (gv && 4 * g + e < nT) mrow[4 * g + e] = sel[e] ? 1 : 0;
+            }
+        }
     }
+}
+
+template <int W, int LOADS>
+veda_status launch_topk_w(const TopkParams& prm, cudaStream_t s) {
+    const size_t smem = topk_warp_words(prm.nT) * sizeof(uint32_t) * W;
+    cudaError_t err = cudaFuncSetAttribute(topk_kernel<W, LOADS>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return cuda_check(err, "topk smem attribute");
+    const unsigned blocks = (unsigned)((prm.rows + W - 1) / W);
+    topk_kernel<W, LOADS><<<blocks, W * 32, smem, s>>>(prm);
+    return cuda_check(cudaGetLastError(), "topk launch");
 }
 
 }  // namespace
@@ -139,25 +365,12 @@ veda_status launch_topk(const Problem& pr, const float* S, uint8_t* mask, int32_
     prm.rows = (long long)pr.B * pr.H * pr.nT;
     prm.nT = pr.nT;
     prm.k = pr.k;
-    const size_t per_warp = ((size_t)((pr.nT + 3) & ~3) + 256) * sizeof(uint32_t);
-    cudaError_t err;
-    if (pr.nT <= 4096) {
-        constexpr int W = 4;
-        const size_t smem = per_warp * W;
-        err = cudaFuncSetAttribute(topk_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem);
-        if (err != cudaSuccess) return cuda_check(err, "topk smem attribute");
-        const unsigned blocks = (unsigned)((prm.rows + W - 1) / W);
-        topk_kernel<W><<<blocks, W * 32, smem, s>>>(prm);
-    } else {
-        constexpr int W = 1;
-        const size_t smem = per_warp * W;
-        err = cudaFuncSetAttribute(topk_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem);
-        if (err != cudaSuccess) return cuda_check(err, "topk smem attribute");
-        topk_kernel<W><<<(unsigned)prm.rows, 32, smem, s>>>(prm);
-    }
-    return cuda_check(cudaGetLastError(), "topk launch");
+    // four warps (rows) per block up to 4096 tiles (<= 74 KB of shared memory),
+    // one above (<= 66 KB at the 16384-tile limit); eight loads in flight per
+    // lane cover a row of up to 1024 scores in one round
+    if (pr.nT <= 1024) return launch_topk_w<4, 8>(prm, s);
+    if (pr.nT <= 4096) return launch_topk_w<4, 16>(prm, s);
+    return launch_topk_w<1, 16>(prm, s);
 }
 
 }  // namespace veda

@@ -29,6 +29,14 @@ veda_status cuda_check(cudaError_t err, const char* what) {
     return fail(VEDA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(err));
 }
 
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+        return 1;
+    return n;
+}
+
 veda_status check_ptr(const void* ptr, const char* name, bool nullable) {
     if (ptr == nullptr) {
         if (nullable) return VEDA_OK;
