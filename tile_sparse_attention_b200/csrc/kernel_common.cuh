@@ -48,7 +48,7 @@ __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity, const 
     }
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast and the
+// Warp-uniform bounded wait: lane 0 polls, the outcome is broadcast and the
 // warp re-converges (the thread sync orders the other lanes after the wait).
 template <class P>
 __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity, const P& p,
