@@ -346,9 +346,33 @@ def run_veda(args, w, world, rank, local):
         _barrier(world)
         e_ms = _max_over_ranks(a.elapsed_time(b) / n_e2e, world)
         h2d = sum(x.numel() * x.element_size() for x in (hostQ, hostK, hostV, hostWq, hostWk))
+        d2h = hostO.numel() * hostO.element_size()
+
+        # the host link alone: plain pinned copies of the same bytes, one
+        # direction at a time, on the same stream; the layer end to end can be
+        # no faster than the slower direction
+        def copy_ms(fn, reps=2):
+            fn()
+            torch.cuda.synchronize(dev)
+            a2, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a2.record(stream)
+            for _ in range(reps):
+                fn()
+            b2.record(stream)
+            torch.cuda.synchronize(dev)
+            return a2.elapsed_time(b2) / reps
+
+        def h2d_copy():
+            for d_, h_ in ((dQ, hostQ), (dK, hostK), (dV, hostV), (dWq, hostWq), (dWk, hostWk)):
+                d_.copy_(h_, non_blocking=True)
+
+        h2d_ms = copy_ms(h2d_copy)
+        d2h_ms = copy_ms(lambda: hostO.copy_(O, non_blocking=True))
+        floor_ms = max(h2d_ms, d2h_ms)
         e2e = {"value": _job_tflops(flops, e_ms, world), "unit": "TFLOP/s",
-               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": hostO.numel() * hostO.element_size()}
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "link": {"h2d_GB_s": h2d / h2d_ms / 1e6, "d2h_GB_s": d2h / d2h_ms / 1e6,
+                        "floor_ms": floor_ms, "frac": floor_ms / e_ms}}
         del hostQ, hostK, hostV, hostO, dQ, dK, dV
 
     cpu = None
