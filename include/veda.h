@@ -177,7 +177,11 @@ veda_status veda_mask_fused(const veda_problem* p, const float* statsQ, const fl
  *   ws : device workspace of at least VEDA_STATUS_BYTES bytes
  * bf16 tensor-core products with fp32 accumulation and an fp32 softmax; P is
  * rounded to bf16 before the P.V product.  An out-of-range index is replaced
- * by tile 0 and reported as VEDA_ERR_BAD_INDEX in the status word.
+ * by tile 0 and reported as VEDA_ERR_BAD_INDEX in the status word.  With the
+ * environment variable VEDA_DEBUG_CHECKS set (not "0"), every row is checked
+ * on the device first and a row with an out-of-range or repeated entry is
+ * also reported as VEDA_ERR_BAD_INDEX (a repeated tile would otherwise be
+ * counted twice).
  */
 veda_status veda_sparse_attn(const veda_problem* p, const uint16_t* Q, const uint16_t* K,
                              const uint16_t* V, const int32_t* idx, uint16_t* O, float* lse,

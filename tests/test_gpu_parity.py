@@ -205,6 +205,28 @@ def test_bad_index_reported(vb):
     assert vb.veda_get_status(ws) == 7  # VEDA_ERR_BAD_INDEX
 
 
+def test_repeated_index_reported_under_debug_checks(vb, monkeypatch):
+    """A row listing one tile twice is in range, so only the optional device-side
+    check (VEDA_DEBUG_CHECKS) can report it; a clean list stays clean under it."""
+    w = workloads.custom("dup", 1, 2, 128, (2, 8, 16), [(1, 8, 16)], 2)
+    t = _inputs(w, "cuda")
+    prob = vb.Problem.from_workload(w)
+    clean = torch.tensor([[0, 1], [1, 0]], dtype=torch.int32).reshape(1, 1, w.nT, 2)
+    clean = clean.expand(1, w.H, w.nT, 2).contiguous().cuda()
+    dup = clean.clone()
+    dup[0, 1, 1] = torch.tensor([1, 1], dtype=torch.int32)
+    O = torch.empty_like(t["Q"])
+    ws = vb.alloc_workspace(prob)
+    monkeypatch.delenv("VEDA_DEBUG_CHECKS", raising=False)
+    vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], dup, O, None, ws)
+    assert vb.veda_get_status(ws) == 0  # not detected without the check
+    monkeypatch.setenv("VEDA_DEBUG_CHECKS", "1")
+    vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], dup, O, None, ws)
+    assert vb.veda_get_status(ws) == 7  # VEDA_ERR_BAD_INDEX
+    vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], clean, O, None, ws)
+    assert vb.veda_get_status(ws) == 0
+
+
 # ------------------------------------------------------------------ whole layer
 def _forward(vb, w, t, want_mask=True):
     prob = vb.Problem.from_workload(w)

@@ -35,6 +35,13 @@ veda_status check_ptr(const void* ptr, const char* name, bool nullable = false);
 veda_status cuda_check(cudaError_t err, const char* what);
 // SMs of the current device (1 if the query fails).
 int sm_count();
+// VEDA_DEBUG_CHECKS set (and not "0"): index lists passed to veda_sparse_attn
+// are validated on the device first (index_check.cu).
+bool debug_checks_enabled();
+// Reports any row of idx [rows, k] with an entry outside [0, nT) or a repeated
+// entry as VEDA_ERR_BAD_INDEX in *status (index_check.cu).
+veda_status launch_check_index(const int32_t* idx, long long rows, int k, int nT, int* status,
+                               cudaStream_t s);
 
 // Launchers (defined next to their kernels).  Each returns VEDA_OK or an
 // error after checking the launch.

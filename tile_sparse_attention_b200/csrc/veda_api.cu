@@ -275,6 +275,9 @@ veda_status veda_sparse_attn(const veda_problem* p, const uint16_t* Q, const uin
     int* status = static_cast<int*>(ws);
     if ((st = cuda_check(cudaMemsetAsync(status, 0, sizeof(int), s), "status reset"))) return st;
     const int k = idx ? pr.k : pr.nT;
+    if (idx != nullptr && debug_checks_enabled() &&
+        (st = launch_check_index(idx, (long long)pr.B * pr.H * pr.nT, k, pr.nT, status, s)))
+        return st;
     return launch_sparse_attn(pr, Q, K, V, idx, k, O, lse, status, s);
 }
 
