@@ -93,3 +93,72 @@ def test_workspace_size_matches_layout(lib):
     r256 = lambda x: (x + 255) // 256 * 256
     want = 256 + 2 * r256(proj) + 2 * r256(stats) + r256(S) + r256(idx)
     assert vb.veda_workspace_size(prob) == want
+
+
+# Every entry point that takes device buffers, with each required pointer in
+# turn made NULL (VEDA_ERR_INVALID_ARG = 1) and each device pointer made
+# misaligned (VEDA_ERR_ALIGN = 4).  The other pointers are a fake, 16-byte
+# aligned address that is never dereferenced: validation fails before any
+# copy or launch, and on a machine without a GPU a CUDA call would have
+# returned VEDA_ERR_CUDA (5) instead.
+#   D required device pointer   N nullable device pointer
+#   H required host pointer     h nullable host pointer (left NULL)
+#   C host candidate tilings    i / f: an integer / float argument
+ENTRY_POINTS = {
+    "veda_tripool": "PDDDDs",
+    "veda_tile_score": "PDDDDDDs",
+    "veda_topk_mask": "PDNDs",
+    "veda_mask_fused": "PDDDDNDDs",
+    "veda_sparse_attn": "PDDDNDNDs",
+    "veda_forward": "PDDDDDDNNNDs",
+    "veda_forward_host": "PHHHHHHhDDDDDDNDis",
+    "veda_tile_search": "PCiDDDDDDDDDDs",
+    "veda_teacher": "PDDDDDDDs",
+    "veda_tile_recall": "PDDNDDs",
+    "veda_distill_kl": "PDDDDDDfDDDDs",
+    "veda_tile_score_noalloc": "PDDDDDs",
+}
+FAKE, MISALIGNED = 0x10000, 0x10008
+
+
+def _entry_args(vb, spec, bad=None, how=None):
+    prob = _problem(vb)  # grid 4x16x32, tiles (2,8,8): nT = 16, k = 3
+    cands = (ctypes.c_int32 * 3)(2, 8, 8)
+    args = []
+    for i, kind in enumerate(spec):
+        if i == bad:
+            args.append(None if how == "null" else ctypes.c_void_p(MISALIGNED))
+        elif kind == "P":
+            args.append(ctypes.byref(prob.c))
+        elif kind == "C":
+            args.append(ctypes.cast(cands, ctypes.c_void_p))
+        elif kind == "i":
+            args.append(1)
+        elif kind == "f":
+            args.append(1.0)
+        elif kind in "sh":
+            args.append(None)
+        else:
+            args.append(None if kind == "N" else ctypes.c_void_p(FAKE))
+    return prob, cands, args
+
+
+@pytest.mark.parametrize("name", sorted(ENTRY_POINTS))
+def test_every_entry_point_rejects_bad_pointers_before_launch(lib, name):
+    import torch
+    import tile_sparse_attention_b200 as vb
+    if torch.cuda.is_available():
+        # the fake addresses must never reach a device: this check runs where
+        # no GPU is visible, so a call that got past validation fails with
+        # VEDA_ERR_CUDA instead of launching
+        pytest.skip("uses fake device addresses; runs only without a visible GPU")
+    spec = ENTRY_POINTS[name]
+    fn = getattr(lib, name)
+    for i, kind in enumerate(spec):
+        if kind in "DHC":
+            _, _, args = _entry_args(vb, spec, bad=i, how="null")
+            assert fn(*args) == 1, f"{name}: NULL argument {i}"
+            assert lib.veda_last_error()
+        if kind in "DN":
+            _, _, args = _entry_args(vb, spec, bad=i, how="misaligned")
+            assert fn(*args) == 4, f"{name}: misaligned argument {i}"
