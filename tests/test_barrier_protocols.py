@@ -1,0 +1,311 @@
+"""Barrier protocols of the two attention kernels, checked by random interleaving.
+
+The tile-skipping attention kernels (sparse_attn.cu: one CTA per query tile;
+sparse_attn_persistent.cu: persistent CTAs looping over query tiles with one
+key-tile stream) hand work between a TMA producer thread, one tcgen05-issuing
+thread and four softmax warps through mbarriers waited on by phase parity.
+This module models those protocols -- the roles, the barriers and their arrival
+counts, a tensor pipe that executes in issue order, copies that land in any
+order -- and runs them under many random interleavings, checking that
+
+* every role finishes (no deadlock);
+* no wait trails its barrier by two completions (the parity would alias);
+* every product reads what it should: the ring stage holds K_g / V_g, the
+  S/P buffer holds S_g / P_g, tensor memory holds Q of the right query tile;
+* a query tile's output accumulator is read by the epilogue only after its
+  last P V product, and before the next tile's first one overwrites it.
+
+It models the kernels' protocol, not their code: a change to the barriers of
+a kernel has to be made here as well.  A planted mistake (a producer that
+refills a ring stage without waiting for its release) must trip a check.
+"""
+import random
+
+import pytest
+
+
+class Bar:
+    """An mbarrier: `count` arrivals complete a phase; `done` counts completions."""
+
+    def __init__(self, count):
+        self.count = count
+        self.pending = count
+        self.done = 0
+
+    def arrive(self):
+        self.pending -= 1
+        assert self.pending >= 0, "more arrivals than the barrier's count"
+        if self.pending == 0:
+            self.done += 1
+            self.pending = self.count
+
+
+def passed(bar, c):
+    """A wait for completion number c of `bar` (the kernels wait on parity c & 1)."""
+    assert bar.done <= c + 1, f"wait for completion {c} trails the barrier ({bar.done} done)"
+    return bar.done >= c + 1
+
+
+def run(roles, tma, tc, rnd):
+    """Roles are generators that yield the predicate they wait on.  Each step
+    advances one ready role, lands one pending copy (any of them) or executes
+    the tensor pipe's oldest operation, chosen at random."""
+    waits = {}
+    live = []
+    for r in roles:
+        w = next(r, None)
+        if w is not None:
+            waits[r] = w
+            live.append(r)
+    while live or tma or tc:
+        moves = [r for r in live if waits[r]()]
+        if tma:
+            moves.append("tma")
+        if tc:
+            moves.append("tc")
+        assert moves, "deadlock: no role can proceed"
+        m = rnd.choice(moves)
+        if m == "tma":
+            tma.pop(rnd.randrange(len(tma)))()
+        elif m == "tc":
+            tc.pop(0)()
+        else:
+            w = next(m, None)
+            if w is None:
+                live.remove(m)
+            else:
+                waits[m] = w
+
+
+# ------------------------------------------------------------------ per query tile
+def model_per_tile(k, NS, seed, p_rescale=0.3, release_wait=True):
+    """sparse_attn.cu: Q staged and copied to tensor memory once; a K/V ring of NS
+    stages, each released by one commit after P_j V_j; two S/P buffers; the
+    issuer runs P_j V_j and then Q K_{j+2}^T."""
+    rnd = random.Random(seed)
+    bq, bq_tmem = Bar(1), Bar(4)
+    k_full = [Bar(1) for _ in range(NS)]
+    v_full = [Bar(1) for _ in range(NS)]
+    kv_empty = [Bar(1) for _ in range(NS)]
+    s_full, p_full = [Bar(1), Bar(1)], [Bar(4), Bar(4)]
+    tma, tc = [], []
+    st = {"K": [None] * NS, "V": [None] * NS, "Qs": False, "Qt": [False] * 4,
+          "S": [None, None], "P": [[None, None] for _ in range(4)], "O": 0}
+
+    def producer():
+        def q_landed():
+            st["Qs"] = True
+            bq.arrive()
+        tma.append(q_landed)
+        for j in range(k):
+            s, n = j % NS, j // NS
+            if n > 0 and release_wait:
+                yield lambda: passed(kv_empty[s], n - 1)
+
+            def kl(s=s, j=j):
+                st["K"][s] = j
+                k_full[s].arrive()
+
+            def vl(s=s, j=j):
+                st["V"][s] = j
+                v_full[s].arrive()
+            tma.append(kl)
+            tma.append(vl)
+
+    def issuer():
+        yield lambda: passed(bq_tmem, 0)
+
+        def issue_qk(j):
+            s, b = j % NS, j & 1
+            yield lambda: passed(k_full[s], j // NS)
+
+            def op():
+                assert st["K"][s] == j, "Q K^T read a ring stage that no longer holds its K tile"
+                assert all(st["Qt"]), "Q K^T before Q reached tensor memory"
+                st["S"][b] = j
+            tc.append(op)
+            tc.append(s_full[b].arrive)
+        yield from issue_qk(0)
+        if k > 1:
+            yield from issue_qk(1)
+        for j in range(k):
+            s, b = j % NS, j & 1
+            yield lambda: passed(p_full[b], j >> 1)
+            yield lambda: passed(v_full[s], j // NS)
+
+            def op(j=j, s=s, b=b):
+                assert st["V"][s] == j, "P V read a ring stage that no longer holds its V tile"
+                assert all(st["P"][w][b] == j for w in range(4)), "P V read a stale P buffer"
+                assert st["O"] == j
+                st["O"] = j + 1
+            tc.append(op)
+            tc.append(kv_empty[s].arrive)
+            if j + 2 < k:
+                yield from issue_qk(j + 2)
+
+    def softmax(w):
+        yield lambda: passed(bq, 0)
+        assert st["Qs"]
+        st["Qt"][w] = True
+        bq_tmem.arrive()
+        for j in range(k):
+            b = j & 1
+            yield lambda: passed(s_full[b], j >> 1)
+            assert st["S"][b] == j, "the softmax read a stale S buffer"
+            if j > 0 and rnd.random() < p_rescale:  # O rescale: P_{j-1} V_{j-1} landed first
+                yield lambda: passed(kv_empty[(j - 1) % NS], (j - 1) // NS)
+                assert st["O"] == j
+            st["P"][w][b] = j
+            p_full[b].arrive()
+        yield lambda: passed(kv_empty[(k - 1) % NS], (k - 1) // NS)
+        assert st["O"] == k, "the epilogue read O before the last P V product"
+
+    run([producer(), issuer()] + [softmax(w) for w in range(4)], tma, tc, rnd)
+
+
+# ------------------------------------------------------------------ persistent
+def model_persistent(n_tiles, k, NS, seed, p_rescale=0.3):
+    """sparse_attn_persistent.cu: the CTA's query tiles n = 0..n_tiles-1 form one
+    key-tile stream g = n*k + j for the K/V ring and the two S/P buffers; Q of
+    tile n is staged in shared memory and copied to tensor-memory buffer n & 1
+    (q_full / q_free / q_tmem), Q of tile n+1 right after the last P of tile n,
+    so tile n+1's first products can run during tile n's epilogue."""
+    rnd = random.Random(seed)
+    total = n_tiles * k
+    q_full, q_free = Bar(1), Bar(4)
+    q_tmem = [Bar(4), Bar(4)]
+    k_full = [Bar(1) for _ in range(NS)]
+    v_full = [Bar(1) for _ in range(NS)]
+    kv_empty = [Bar(1) for _ in range(NS)]
+    s_full, p_full = [Bar(1), Bar(1)], [Bar(4), Bar(4)]
+    tma, tc = [], []
+    st = {"K": [None] * NS, "V": [None] * NS, "Qs": None,
+          "Qt": [[None, None] for _ in range(4)], "S": [None, None],
+          "P": [[None, None] for _ in range(4)], "O": (None, 0), "O_read": [-1] * 4}
+
+    def producer():
+        for n in range(n_tiles):
+            if n > 0:
+                yield lambda: passed(q_free, n - 1)
+
+            def q_landed(n=n):
+                st["Qs"] = n
+                q_full.arrive()
+            tma.append(q_landed)
+            for j in range(k):
+                g = n * k + j
+                s, f = g % NS, g // NS
+                if f > 0:
+                    yield lambda: passed(kv_empty[s], f - 1)
+
+                def kl(s=s, g=g):
+                    st["K"][s] = g
+                    k_full[s].arrive()
+
+                def vl(s=s, g=g):
+                    st["V"][s] = g
+                    v_full[s].arrive()
+                tma.append(kl)
+                tma.append(vl)
+
+    def issuer():
+        cnt = {"g": 0, "n": 0, "j": 0}  # the next Q K^T: stream index, query tile, key tile
+
+        def issue_next_qk():
+            g, n = cnt["g"], cnt["n"]
+            s, b = g % NS, g & 1
+            if cnt["j"] == 0:
+                yield lambda: passed(q_tmem[n & 1], n >> 1)
+            yield lambda: passed(k_full[s], g // NS)
+
+            def op():
+                assert st["K"][s] == g, "Q K^T read a ring stage that no longer holds its K tile"
+                assert all(st["Qt"][w][n & 1] == n for w in range(4)), \
+                    "Q K^T read a tensor-memory Q buffer that does not hold its query tile"
+                st["S"][b] = g
+            tc.append(op)
+            tc.append(s_full[b].arrive)
+            cnt["g"] += 1
+            cnt["j"] += 1
+            if cnt["j"] == k:
+                cnt["j"] = 0
+                cnt["n"] += 1
+        if total > 0:
+            yield from issue_next_qk()
+        if total > 1:
+            yield from issue_next_qk()
+        for g in range(total):
+            s, b, n, j = g % NS, g & 1, g // k, g % k
+            yield lambda: passed(p_full[b], g >> 1)
+            yield lambda: passed(v_full[s], g // NS)
+
+            def op(g=g, s=s, b=b, n=n, j=j):
+                assert st["V"][s] == g, "P V read a ring stage that no longer holds its V tile"
+                assert all(st["P"][w][b] == g for w in range(4)), "P V read a stale P buffer"
+                if j == 0:
+                    assert all(r == n - 1 for r in st["O_read"]), \
+                        "the first P V of a tile overwrote O before the epilogue read it"
+                    st["O"] = (n, 1)
+                else:
+                    assert st["O"] == (n, j)
+                    st["O"] = (n, j + 1)
+            tc.append(op)
+            tc.append(kv_empty[s].arrive)
+            if cnt["g"] < total:
+                yield from issue_next_qk()
+
+    def softmax(w):
+        def copy_q(n):
+            yield lambda: passed(q_full, n)
+            assert st["Qs"] == n, "the staging buffer does not hold Q of this tile"
+            st["Qt"][w][n & 1] = n
+            q_tmem[n & 1].arrive()
+            q_free.arrive()
+        if n_tiles > 0:
+            yield from copy_q(0)
+        for n in range(n_tiles):
+            for j in range(k):
+                g = n * k + j
+                b = g & 1
+                yield lambda: passed(s_full[b], g >> 1)
+                assert st["S"][b] == g, "the softmax read a stale S buffer"
+                if j > 0 and rnd.random() < p_rescale:
+                    yield lambda: passed(kv_empty[(g - 1) % NS], (g - 1) // NS)
+                    assert st["O"] == (n, j)
+                st["P"][w][b] = g
+                p_full[b].arrive()
+            if n + 1 < n_tiles:
+                yield from copy_q(n + 1)
+            g_last = n * k + k - 1
+            yield lambda: passed(kv_empty[g_last % NS], g_last // NS)
+            assert st["O"] == (n, k), "the epilogue read O before the tile's last P V product"
+            st["O_read"][w] = n
+
+    run([producer(), issuer()] + [softmax(w) for w in range(4)], tma, tc, rnd)
+
+
+@pytest.mark.parametrize("NS", [2, 3, 4])
+@pytest.mark.parametrize("k", [1, 2, 3, 5, 8])
+def test_per_query_tile_protocol(k, NS):
+    for seed in range(25):
+        model_per_tile(k, NS, seed)
+
+
+@pytest.mark.parametrize("NS", [3, 4])
+@pytest.mark.parametrize("k", [1, 2, 3, 5])
+@pytest.mark.parametrize("n_tiles", [0, 1, 2, 3, 5])
+def test_persistent_protocol(n_tiles, k, NS):
+    for seed in range(12):
+        model_persistent(n_tiles, k, NS, seed)
+
+
+def test_a_planted_refill_race_is_caught():
+    """Without the wait for a stage's release, some interleaving overwrites a K or
+    V tile before its product reads it."""
+    caught = 0
+    for seed in range(40):
+        try:
+            model_per_tile(8, 2, seed, release_wait=False)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
