@@ -212,7 +212,7 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
  *   dWq, dWk  : device fp32 [H, d, d] staging
  *   dlse      : device fp32 [B, H, N] staging, needed when hlse is not NULL
  *   ws        : at least veda_workspace_size() bytes
- *   head_chunk: heads per chunk, 1..H (0 picks H/8, at least 1)
+ *   head_chunk: heads per chunk, 1..H (0 picks 1)
  * Host buffers should be page-locked (cudaHostAlloc / pinned) for the copies
  * to overlap the kernels; with pageable memory the copies are synchronous.
  * When `stream` completes, hO (and hlse) hold the results.  The status word in

@@ -315,7 +315,9 @@ veda_status veda_forward_host(const veda_problem* p, const uint16_t* hQ, const u
         return st;
     if (head_chunk < 0 || head_chunk > pr.H)
         return fail(VEDA_ERR_INVALID_ARG, "head_chunk must be in 0..H");
-    if (head_chunk == 0) head_chunk = pr.H / 8 > 0 ? pr.H / 8 : 1;
+    // default: one head per chunk (the copies bound the layer, and the smallest
+    // chunk shortens the fill and drain of the pipeline the most)
+    if (head_chunk == 0) head_chunk = 1;
     return forward_host_impl(p, pr, hQ, hK, hV, hWq, hWk, hO, hlse, dQ, dK, dV, dWq, dWk, dO,
                              hlse ? dlse : nullptr, ws, head_chunk, (cudaStream_t)stream);
 }
