@@ -6,8 +6,9 @@ a full stable sort.  Tiny inputs only.
 
 Source: "Veda: Scalable Video Diffusion via Distilled Sparse Attention"
 (project page) -- "Attention Structure Distillation" (Teacher, Estimator,
-Execution), "Principle 02 Head-Conditioned Tile Geometry", "Theoretical
-Rationale" 1 (Softmax Geometry) and 2 (Tile Statistics).
+Execution), "Principle 01 Full-Attention Structure Distillation",
+"Principle 02 Head-Conditioned Tile Geometry", "Theoretical Rationale" 1
+(Softmax Geometry), 2 (Tile Statistics) and 4 (Distillation Objective).
 """
 from __future__ import annotations
 
@@ -117,3 +118,22 @@ def teacher(Q, K, grid, shapes, scale):
             per_h.append(P[tok[:, :, None, None], tok[None, None, :, :]].max(axis=(1, 3)))
         out.append(np.stack(per_h))
     return np.stack(out)
+
+
+def distill_kl(statsQ, statsK, Wq, Wk, teacher, tau) -> float:
+    """Distillation loss from its definition ("Theoretical Rationale" 4).
+
+    Per query-tile row: the target distribution is the teacher row divided by
+    its sum, the estimator distribution is softmax(S / tau) over the key tiles,
+    and the row's term is KL(target || estimator) = sum_j t_j log(t_j / p_j),
+    evaluated by scipy's relative entropy (0 where t_j = 0).  The loss is the
+    mean of the row terms over all B*H*nT rows.
+    """
+    from scipy.special import rel_entr, softmax
+
+    S = scores(statsQ, statsK, Wq, Wk)
+    nT = S.shape[-1]
+    pred = softmax(S.reshape(-1, nT) / tau, axis=1)
+    tgt = teacher.reshape(-1, nT) / teacher.reshape(-1, nT).sum(axis=1, keepdims=True)
+    rows = rel_entr(tgt, pred).sum(axis=1)
+    return float(rows.mean())

@@ -47,6 +47,27 @@ MUTANTS = {
         "dWq[(h * d + ci) * d + co] += sq[ci] * dq[s3 * d + co];",
         "dWq[(h * d + ci) * d + co] += sk[ci] * dq[s3 * d + co];"),
     "distillation target not normalised": ("double tg = t[j] / tsum;", "double tg = t[j];"),
+    # reversed divergence KL(estimator || target), with its own consistent
+    # gradient: the chain-rule and finite-difference pins cannot see it
+    "distillation KL reversed (loss and gradient)": (
+        """            if (tg > 0.0) kl += tg * (log(tg) - logp);
+            G[row * nT + j] = (exp(logp) - tg) / (tau * (double)R);
+        }""",
+        """            kl += exp(logp) * (logp - log(tg));
+        }
+        for (int64_t j = 0; j < nT; ++j) {
+            double logp = s[j] / tau - lse;
+            double tg = t[j] / tsum;
+            G[row * nT + j] = exp(logp) * (logp - log(tg) - kl) / (tau * (double)R);
+        }"""),
+    # the row terms summed instead of averaged, gradient scaled to match
+    "distillation sums the rows (loss and gradient)": (
+        """            G[row * nT + j] = (exp(logp) - tg) / (tau * (double)R);
+        }
+        total += kl;""",
+        """            G[row * nT + j] = (exp(logp) - tg) / tau;
+        }
+        total += kl * (double)R;"""),
     "e4m3 ties go to the lower code": ("code = (lo & 1) ? lo + 1 : lo;", "code = lo;"),
     "e4m3 exponent bias 8": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);",
                              "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
@@ -76,6 +97,8 @@ def pin_suite(o):
     yield lambda: pins.test_tile_recall_hand_cases(o)
     yield lambda: pins.test_tile_recall_brute_force(o)
     yield lambda: pins.test_distill_gradient_matches_finite_differences(o, 0.7, 1)
+    yield lambda: pins.test_distill_loss_matches_definition(o, 0.7, 1, 0)
+    yield lambda: pins.test_distill_loss_matches_definition(o, 1.0, 2, 11)
     yield lambda: pins.test_distill_zero_when_target_equals_prediction(o)
     yield lambda: pins.test_distill_invariances_and_positivity(o)
     yield lambda: pins.test_tile_search_brute_force(o)

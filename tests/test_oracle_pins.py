@@ -372,6 +372,23 @@ def test_distill_gradient_matches_finite_differences(oracle, tau, B):
             assert abs(fd - dW[h, a, b]) <= 1e-4 * scale + 1e-10, (side, h, a, b, fd, dW[h, a, b])
 
 
+@pytest.mark.parametrize("tau,B,seed", [(0.7, 1, 0), (1.0, 2, 11), (3.0, 1, 4)])
+def test_distill_loss_matches_definition(oracle, tau, B, seed):
+    """The loss value against the brute-force KL written from the definition:
+    direction KL(target || estimator) and the mean over the B*H*nT rows.  A
+    reversed divergence or a sum over rows changes the value (the teacher rows
+    here are far from the estimator's, so the two directions differ)."""
+    sq, sk, Wq, Wk, T = _distill_case(seed=seed, B=B)
+    L = oracle.distill_kl(sq, sk, Wq, Wk, T, tau, grads=False)
+    ref = bf.distill_kl(sq, sk, Wq, Wk, T, tau)
+    assert abs(L - ref) <= 1e-12 * max(1.0, abs(ref)), (L, ref)
+    # a teacher with zero entries: those terms contribute nothing
+    Tz = T.copy()
+    Tz[..., ::3] = 0.0
+    Lz = oracle.distill_kl(sq, sk, Wq, Wk, Tz, tau, grads=False)
+    assert abs(Lz - bf.distill_kl(sq, sk, Wq, Wk, Tz, tau)) <= 1e-12 * max(1.0, abs(Lz))
+
+
 def test_distill_zero_when_target_equals_prediction(oracle):
     sq, sk, Wq, Wk, _ = _distill_case(seed=3)
     tau = 1.7
