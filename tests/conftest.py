@@ -19,3 +19,18 @@ def pytest_configure(config):
 def oracle():
     from oracle import Oracle
     return Oracle()
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Per mask comparison: rows checked, rows the 1e-3 gap rule exempts, and
+    rows identical to the oracle's (printed even under -q)."""
+    try:
+        import parity_helpers
+    except Exception:
+        return
+    if not parity_helpers.MASK_REPORT:
+        return
+    terminalreporter.write_line("mask rows (label: rows, exempt by the gap rule, identical):")
+    for label, rows, n_ex, n_exact in parity_helpers.MASK_REPORT:
+        terminalreporter.write_line(f"  {label}: {rows}, {n_ex} ({100.0 * n_ex / rows:.1f}%), "
+                                    f"{n_exact} ({100.0 * n_exact / rows:.2f}%)")

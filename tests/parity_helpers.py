@@ -87,9 +87,29 @@ def exempt_rows(S_ora: np.ndarray, k: int) -> np.ndarray:
     return (gap <= GAP_REL * np.maximum(np.abs(sk), np.abs(sk1))).reshape(S_ora.shape[:-1])
 
 
+# One line per mask comparison of the session: (label, rows, exempt rows,
+# rows identical to the oracle's).  tests/conftest.py prints it at the end.
+MASK_REPORT = []
+
+# Ceilings and floors, measured on the seeded inputs (CPU draws) with a margin.
+# The 1e-3 gap rule exempts many rows, because neighbouring tiles have close
+# scores: 23-29% at 480P / 720P, 59% at long video, 2-84% across the sweep (the
+# most at T = 64, s <= 80%).  What bounds the claim instead is the floor on rows
+# identical to the oracle's, exempt or not: an fp32 score agrees with the fp64
+# one on >= 99.86% of the rows at every size (the GPU's three-term TF32 score is
+# as accurate as fp32), so at least 99% must be identical.
+MAX_EXEMPT_FRAC = 0.9
+MIN_EXACT_FRAC = 0.99
+
+
 def check_masks(mask_gpu: np.ndarray, idx_gpu: np.ndarray, S_ora: np.ndarray, mask_ora, idx_ora,
-                k: int):
-    """Bit-exact on non-exempt rows; exempt rows: k ones and every clear winner kept."""
+                k: int, label: str = "", max_exempt_frac: float = MAX_EXEMPT_FRAC,
+                min_exact_frac: float = MIN_EXACT_FRAC):
+    """Bit-exact on non-exempt rows; exempt rows: k ones and every clear winner kept.
+
+    Also bounds how much the gap rule exempts (at most ``max_exempt_frac`` of
+    the rows) and how many rows, exempt or not, must equal the oracle's row
+    exactly (at least ``min_exact_frac``); returns the exempt-row count."""
     ex = exempt_rows(S_ora, k)
     nT = S_ora.shape[-1]
     assert np.all(mask_gpu.sum(-1) == k)
@@ -103,7 +123,14 @@ def check_masks(mask_gpu: np.ndarray, idx_gpu: np.ndarray, S_ora: np.ndarray, ma
         sk = -np.sort(-flat_S[r])[k - 1]
         clear = flat_S[r] > sk + GAP_REL * abs(sk)
         assert np.all(flat_m[r][clear] == 1)
-    return int(ex.sum())
+    rows = int(ex.size)
+    n_ex = int(ex.sum())
+    n_exact = int(np.all(mask_gpu.reshape(-1, nT) == np.asarray(mask_ora).reshape(-1, nT),
+                         axis=1).sum())
+    MASK_REPORT.append((label or f"nT={nT} k={k}", rows, n_ex, n_exact))
+    assert n_ex <= max_exempt_frac * rows, f"{label}: {n_ex} of {rows} rows exempt"
+    assert n_exact >= min_exact_frac * rows, f"{label}: only {n_exact} of {rows} rows exact"
+    return n_ex
 
 
 def check_attention(O_gpu_bits: np.ndarray, lse_gpu: np.ndarray, units, O_ora, lse_ora, toks):

@@ -76,7 +76,7 @@ def test_mask_with_fp8_weights(vb, oracle):
     heads = list(range(H))
     ora = ph.oracle_mask_prep_heads(oracle, w, Qb, Kb, Wq_o, Wk_o, heads)
     ph.check_masks(g["mask"].cpu().numpy(), g["idx"].cpu().numpy(), ora["S"], ora["mask"],
-                   ora["idx"], w.k)
+                   ora["idx"], w.k, label=f"fp8 weights {w.name}")
     # tile recall of the fp8-weight mask against the fp32-weight mask (GPU kernel
     # against the oracle's count on the same index lists)
     g32 = ph.gpu_mask_prep(vb, prob, t["Q"], t["K"], t["Wq"], t["Wk"])

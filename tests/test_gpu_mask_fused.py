@@ -94,7 +94,7 @@ def test_fused_against_oracle(vb, oracle, make, heads):
     Wq, Wk = t["Wq"].cpu().numpy(), t["Wk"].cpu().numpy()
     ora = ph.oracle_mask_prep_heads(oracle, w, Qb, Kb, Wq, Wk, heads)
     ph.check_masks(mf[:, heads].cpu().numpy(), i_f[:, heads].cpu().numpy(), ora["S"],
-                   ora["mask"], ora["idx"], w.k)
+                   ora["mask"], ora["idx"], w.k, label=f"fused {w.name}")
 
 
 def test_fused_exact_ties_and_zero_scores(vb, oracle):

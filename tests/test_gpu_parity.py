@@ -55,7 +55,7 @@ def test_tripool_and_score_parity(vb, oracle, make, heads):
     err = np.abs(S_gpu - ora["S"])
     assert np.all(err <= bound), f"score error {err.max()} (bound {bound.min()})"
     ph.check_masks(g["mask"][:, heads].cpu().numpy(), g["idx"][:, heads].cpu().numpy(),
-                   ora["S"], ora["mask"], ora["idx"], w.k)
+                   ora["S"], ora["mask"], ora["idx"], w.k, label=f"mask prep {w.name}")
 
 
 def test_topk_bit_exact_on_given_scores(vb, oracle):
@@ -252,7 +252,7 @@ def _forward_parity(vb, oracle, w, heads, per_head, device="cuda"):
     ora = oracle.mask_prep(Qb, Kb, Wq, Wk, w.grid, shapes, w.k)
     idx_g = idx.index_select(1, sel).cpu().numpy()
     ph.check_masks(mask.index_select(1, sel).cpu().numpy(), idx_g, ora["S"], ora["mask"],
-                   ora["idx"], w.k)
+                   ora["idx"], w.k, label=f"forward {w.name}")
     # attention on sampled query tiles; the oracle gets the (verified) GPU index list
     units = workloads.sample_units(w, per_head, seed=4)
     hmap = {h: n for n, h in enumerate(heads)}
