@@ -41,11 +41,38 @@ import workloads  # noqa: E402
 METRIC = "ms/layer and effective TFLOP/s of tile-sparse attention (+mask prep) at 95% sparsity"
 
 
-# DRAM bytes (read + write) of one attention launch, from one ncu capture of
-# dram__bytes_read.sum + dram__bytes_write.sum on this kernel version (profile
-# summary: profiles/launches_long_video_245k.md).  Emptied whenever the kernel
-# changes, until the counters are taken again.
-ATTN_DRAM_BYTES = {"long_video_245k": 3.41e9 + 2.02e9}
+# DRAM bytes (read + write) of one attention launch on the estimator's mask,
+# from one ncu capture of dram__bytes_read.sum + dram__bytes_write.sum, with the
+# kernel version it was taken on.  A kernel change empties the entry until the
+# counters are taken again.
+ATTN_DRAM_BYTES = {"long_video_245k": {"bytes": 3.41e9 + 2.02e9,
+                                       "kernel": "sparse_attn_kernel<128,128,3>, commit 2b2780b",
+                                       "capture": "ncu --metrics dram__bytes_read.sum,"
+                                                  "dram__bytes_write.sum, one launch"}}
+
+
+def _config(w, world):
+    """The `config` object of both arms' JSON lines."""
+    return dict(w.describe(),
+                parallelism="replicas (one layer per GPU)" if world > 1 else "single GPU",
+                l2=f"inputs larger than L2 (Q/K/V {3 * w.B * w.H * w.N * w.d * 2 / 1e9:.2f} GB)")
+
+
+def key_tile_coverage(idx, nT):
+    """Per (b, h): distinct key tiles the index lists select, and the share of
+    all selections that fall on the k most-selected key tiles (how strongly the
+    rows concentrate on a few key tiles, i.e. how much of K/V stays in L2)."""
+    BH = idx.shape[0] * idx.shape[1]
+    flat = idx.reshape(BH, -1).long()
+    counts = torch.zeros((BH, nT), dtype=torch.int64, device=idx.device)
+    counts.scatter_add_(1, flat, torch.ones_like(flat))
+    distinct = (counts > 0).sum(1).double()
+    k = idx.shape[-1]
+    top = counts.sort(1, descending=True).values[:, :k].sum(1).double() / flat.shape[1]
+    return {"distinct_key_tiles_per_head": {"mean": distinct.mean().item(),
+                                            "min": distinct.min().item(),
+                                            "max": distinct.max().item(), "of": nT},
+            "share_of_selections_on_top_k_tiles": top.mean().item()}
 
 
 def _peaks():
@@ -213,7 +240,7 @@ def run_reference(args, w, world, rank):
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": dict(w.describe(), parallelism="replicas"),
+            "data": "synthetic", "config": _config(w, world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"],
                              "kind": "oracle", "sample": res["sample"]},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -388,15 +415,15 @@ def run_veda(args, w, world, rank, local):
                "full_layer_s_extrapolated": res["full_layer_s"]}
 
     if rank == 0:
-        peak = peaks["bf16_sus"]
+        # the attention kernel is timed per launch (~50 ms): the burst peak applies
+        peak = peaks["bf16"]
+        traffic = ATTN_DRAM_BYTES.get(w.name)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": dict(w.describe(), parallelism="replicas (one layer per GPU)" if world > 1
-                           else "single GPU",
-                           l2=f"inputs larger than L2 (Q/K/V {3 * B * H * N * d * 2 / 1e9:.2f} GB)"),
+            "config": _config(w, world),
             "ms_per_layer": ms,
             "frac_of_peak": {"measured_bf16_burst": value / world / peaks["bf16"],
                              "measured_bf16_sustained": value / world / peaks["bf16_sus"],
@@ -404,10 +431,14 @@ def run_veda(args, w, world, rank, local):
                              "peaks": peaks["source"]},
             "roofline": {"bound": "tensor", "kernel": "sparse_attn", "achieved": attn_tf,
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
-                         "peak_kind": "bf16 sustained (" + peaks["source"] + ")",
-                         "frac_of_burst": attn_tf / peaks["bf16"],
-                         "traffic": ATTN_DRAM_BYTES.get(w.name),
+                         "peak_kind": "bf16 burst (" + peaks["source"] + "), the kernel is "
+                                      "timed per launch",
+                         "frac_of_sustained": attn_tf / peaks["bf16_sus"],
+                         "traffic": traffic["bytes"] if traffic else None,
+                         "traffic_source": ({"kernel": traffic["kernel"],
+                                             "capture": traffic["capture"]} if traffic else None),
                          "algorithmic_flops_per_launch": flops},
+            "estimator_mask": key_tile_coverage(idx, nT),
             "kernels_ms": per,
             "mask_prep": mask_prep,
             "dense_path": {"attn_ms": dense_ms,
@@ -420,6 +451,90 @@ def run_veda(args, w, world, rank, local):
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- mask kinds
+def random_index_lists(w, device, seed=1):
+    """Seeded index lists: per row, k distinct key tiles drawn uniformly, ascending."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    rows = w.B * w.H * w.nT
+    out = torch.empty((rows, w.k), dtype=torch.int32, device=device)
+    for r0 in range(0, rows, 8192):
+        r1 = min(rows, r0 + 8192)
+        u = torch.rand((r1 - r0, w.nT), generator=g, device=device)
+        out[r0:r1] = u.topk(w.k, dim=1).indices.sort(dim=1).values.int()
+    return out.view(w.B, w.H, w.nT, w.k)
+
+
+def local_index_lists(w, device):
+    """Per query tile, the k key tiles whose centres are nearest in (t, y, x)
+    token coordinates (squared Euclidean distance, ties to the lower index):
+    the spatio-temporal locality of video attention, ascending."""
+    out = torch.empty((w.B, w.H, w.nT, w.k), dtype=torch.int32, device=device)
+    for shape in sorted(set(w.tile_shapes)):
+        pt, ph, pw = shape
+        nh, nw = w.Hs // ph, w.Ws // pw
+        j = torch.arange(w.nT, device=device, dtype=torch.int64)
+        c = torch.stack([2 * (j // (nh * nw)) * pt + pt, 2 * ((j // nw) % nh) * ph + ph,
+                         2 * (j % nw) * pw + pw], 1)  # doubled centres: integers
+        lists = torch.empty((w.nT, w.k), dtype=torch.int32, device=device)
+        for i0 in range(0, w.nT, 256):
+            i1 = min(w.nT, i0 + 256)
+            d2 = ((c[i0:i1, None, :] - c[None, :, :]) ** 2).sum(-1)
+            key = d2 * w.nT + j[None, :]
+            lists[i0:i1] = key.topk(w.k, dim=1, largest=False).indices.sort(dim=1).values.int()
+        for h, sh in enumerate(w.tile_shapes):
+            if sh == shape:
+                out[:, h] = lists
+    return out
+
+
+def run_masks(args, w):
+    """Attention alone on three kinds of index list at the same k: the
+    estimator's mask (as in the layer), seeded uniformly random rows (every key
+    tile in use, little reuse in L2) and the k nearest tiles in (t, y, x).  One
+    JSON line per kind: time, effective TFLOP/s, fraction of the burst peak,
+    key-tile coverage, clocks."""
+    import tile_sparse_attention_b200 as vb
+    vb.load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = _peaks()
+    t = workloads.generate(w, device=dev)
+    prob = vb.Problem.from_workload(w)
+    B, H, N, d, nT, k = w.B, w.H, w.N, w.d, w.nT, w.k
+    ws = vb.alloc_workspace(prob, dev)
+    est = torch.empty((B, H, nT, k), dtype=torch.int32, device=dev)
+    vb.veda_forward(prob, t["Q"], t["K"], t["V"], t["Wq"], t["Wk"], torch.empty_like(t["Q"]),
+                    None, est, None, ws)
+    kinds = {"estimator": est, "random": random_index_lists(w, dev), "local": local_index_lists(w, dev)}
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    flops = w.sparse_flops()
+    reps = max(3, args.steps)
+    for name, idx in kinds.items():
+        fn = lambda: vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O, lse, ws)
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        with ClockSampler(0) as clk:
+            for r in range(reps):
+                evs[r].record(stream)
+                fn()
+            evs[reps].record(stream)
+            torch.cuda.synchronize(dev)
+        ms = statistics.median(evs[r].elapsed_time(evs[r + 1]) for r in range(reps))
+        tf = flops / (ms * 1e-3) / 1e12
+        print(json.dumps({"row": "attention by mask kind", "mask": name, "workload": w.name,
+                          "k": k, "launches": reps, "ms_median": ms, "TFLOP_s": tf,
+                          "frac_bf16_burst": tf / peaks["bf16"],
+                          "frac_bf16_sustained": tf / peaks["bf16_sus"],
+                          "coverage": key_tile_coverage(idx, nT), "clocks": clk.summary(),
+                          "status": vb.veda_get_status(ws)}), flush=True)
     return 0
 
 
@@ -472,9 +587,10 @@ def run_sweep(args):
                 vb.veda_topk_mask(prob, S, None, idx)
                 vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O, lse, ws)
             reps = 3 if w.k * nT <= 400_000 else 2
-            ms = timed(layer, reps)
-            attn_ms = timed(lambda: vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O, lse,
-                                                        ws), reps)
+            with ClockSampler(0) as clk:
+                ms = timed(layer, reps)
+                attn_ms = timed(lambda: vb.veda_sparse_attn(prob, t["Q"], t["K"], t["V"], idx, O,
+                                                            lse, ws), reps)
             print(json.dumps({"row": "sweep", "workload": w.name, "T": T, "tokens": N, "tiles": nT,
                               "sparsity_pct": sp, "k": w.k, "ms_per_layer": ms, "attn_ms": attn_ms,
                               "TFLOP_s": w.sparse_flops() / (ms * 1e-3) / 1e12,
@@ -482,7 +598,8 @@ def run_sweep(args):
                               "attn_frac_bf16_burst": w.sparse_flops() / (attn_ms * 1e-3) / 1e12
                               / peaks["bf16"],
                               "dense_attn_ms": dense_ms, "speedup_attention": dense_ms / attn_ms,
-                              "speedup_layer": dense_ms / ms, "status": vb.veda_get_status(ws)}),
+                              "speedup_layer": dense_ms / ms, "clocks": clk.summary(),
+                              "status": vb.veda_get_status(ws)}),
                   flush=True)
             del ws, idx
         del t, statsQ, statsK, S, O, lse
@@ -617,6 +734,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time the sweep points (T x sparsity) instead")
+    ap.add_argument("--masks", action="store_true",
+                    help="time the attention alone on estimator, random and local index lists")
     ap.add_argument("--rows", default="",
                     help="comma list of f1,f2,f3,f4: time the next rows instead")
     args = ap.parse_args()
@@ -631,6 +750,8 @@ def main():
         return run_sweep(args)
     if args.rows:
         return run_rows(args, w, set(args.rows.split(",")))
+    if args.masks:
+        return run_masks(args, w)
     world, rank, local = _dist_init()
     try:
         if args.impl == "reference":

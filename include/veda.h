@@ -217,6 +217,12 @@ veda_status veda_forward(const veda_problem* p, const uint16_t* Q, const uint16_
  * to overlap the kernels; with pageable memory the copies are synchronous.
  * When `stream` completes, hO (and hlse) hold the results.  The status word in
  * ws covers every chunk (veda_get_status).
+ * Exception to the rule that a failed call has launched nothing: an error met
+ * after the first chunk's copies were queued (a CUDA call failing mid-way) is
+ * returned after `stream` has been made to wait for every copy already queued
+ * (or, if that fails too, after those copies finished), so once `stream`
+ * completes no copy of this call reads or writes the host buffers; the earlier
+ * chunks' kernels and copies may have run.
  */
 veda_status veda_forward_host(const veda_problem* p, const uint16_t* hQ, const uint16_t* hK,
                               const uint16_t* hV, const float* hWq, const float* hWk,
@@ -304,7 +310,7 @@ veda_status veda_distill_kl(const veda_problem* p, const float* statsQ, const fl
 veda_status veda_get_status(const void* ws, veda_stream_t stream, int32_t* device_status);
 
 /*
- * The paper has no counterpart for the two calls below; they exist for
+ * The paper has no counterpart for the calls below; they exist for
  * callers that cannot allocate device memory (an application that only
  * receives device pointers for its inputs and outputs from another runtime, a
  * plugin whose host forbids allocations after start-up, a real-time loop that
@@ -328,6 +334,16 @@ size_t veda_noalloc_scratch_bytes(void);
 veda_status veda_tile_score_noalloc(const veda_problem* p, const float* statsQ,
                                     const float* statsK, const float* Wq, const float* Wk,
                                     float* S, veda_stream_t stream);
+
+/*
+ * No counterpart in the paper either.  Waits for `stream`, then copies the
+ * status word that the last veda_tile_score_noalloc call on the current device
+ * left in the fixed array into *device_status: VEDA_OK, or VEDA_ERR_TIMEOUT if
+ * a bounded wait of the score kernel gave up (that call's S is then
+ * incomplete).  The same race as above applies: a later or overlapping call
+ * clears and reuses the word.  VEDA_ERR_INVALID_ARG if device_status is NULL.
+ */
+veda_status veda_noalloc_get_status(veda_stream_t stream, int32_t* device_status);
 
 #ifdef __cplusplus
 }

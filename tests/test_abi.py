@@ -117,6 +117,7 @@ ENTRY_POINTS = {
     "veda_tile_recall": "PDDNDDs",
     "veda_distill_kl": "PDDDDDDfDDDDs",
     "veda_tile_score_noalloc": "PDDDDDs",
+    "veda_noalloc_get_status": "sH",
 }
 FAKE, MISALIGNED = 0x10000, 0x10008
 

@@ -19,8 +19,8 @@ def vb():
     return m
 
 
-def _run(vb, w, head_chunk):
-    t = {n: v.cuda() for n, v in workloads.generate(w, device="cpu").items()}
+def _run(vb, w, head_chunk, draw="cpu"):
+    t = {n: v.cuda() for n, v in workloads.generate(w, device=draw).items()}
     prob = vb.Problem.from_workload(w)
     B, H, N, d = w.B, w.H, w.N, w.d
     ws = vb.alloc_workspace(prob)
@@ -53,6 +53,12 @@ def _run(vb, w, head_chunk):
 ])
 def test_forward_host_equals_forward(vb, name, make, chunk):
     _run(vb, make(), chunk)
+
+
+def test_forward_host_long_video_default_chunk(vb):
+    """The benchmarked end-to-end call: 245,760 tokens, 32 heads, 6 GB of host
+    input, the default of one head per chunk (inputs drawn on the device)."""
+    _run(vb, workloads.long_video(), 0, draw="cuda")
 
 
 def test_forward_host_rejects_bad_chunk(vb):

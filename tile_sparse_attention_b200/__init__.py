@@ -96,6 +96,8 @@ def load_library(path: str = LIB_PATH):
     lib.veda_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.veda_tile_score_noalloc.argtypes = [ctypes.POINTER(veda_problem)] + [_P] * 6
     lib.veda_tile_score_noalloc.restype = st
+    lib.veda_noalloc_get_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
+    lib.veda_noalloc_get_status.restype = st
     _lib = lib
     return lib
 
@@ -332,6 +334,15 @@ def veda_tile_score_noalloc(problem: Problem, statsQ, statsK, Wq, Wk, S, stream=
 
 def veda_noalloc_scratch_bytes() -> int:
     return int(load_library().veda_noalloc_scratch_bytes())
+
+
+def veda_noalloc_get_status(stream=None) -> int:
+    """Device status word of the last veda_tile_score_noalloc call on the current
+    device (0, or VEDA_ERR_TIMEOUT when a bounded wait gave up); waits for the
+    stream first."""
+    out = ctypes.c_int32(0)
+    _check(load_library().veda_noalloc_get_status(_stream(stream), ctypes.byref(out)))
+    return int(out.value)
 
 
 def alloc_workspace(problem: Problem, device="cuda") -> torch.Tensor:

@@ -78,6 +78,23 @@ veda_status forward_host_impl(const veda_problem* p, const Problem& pr, const ui
     if ((st = cuda_check(cudaStreamWaitEvent(cs.in, entry, 0), "stream wait"))) return st;
     if ((st = cuda_check(cudaStreamWaitEvent(cs.out, entry, 0), "stream wait"))) return st;
     if ((st = cuda_check(cudaMemsetAsync(ws, 0, sizeof(int), s), "status reset"))) return st;
+    // From here on copies may be queued on the copy streams: an error return
+    // first makes the caller's stream wait for them (or, if even that fails,
+    // waits on the host), so no copy touches the caller's buffers after the
+    // caller's stream has completed.
+    auto fail_joined = [&](veda_status err) -> veda_status {
+        cudaEvent_t ein = nullptr, eout = nullptr;
+        bool joined = events.make(&ein) == VEDA_OK && events.make(&eout) == VEDA_OK &&
+                      cudaEventRecord(ein, cs.in) == cudaSuccess &&
+                      cudaEventRecord(eout, cs.out) == cudaSuccess &&
+                      cudaStreamWaitEvent(s, ein, 0) == cudaSuccess &&
+                      cudaStreamWaitEvent(s, eout, 0) == cudaSuccess;
+        if (!joined) {
+            cudaStreamSynchronize(cs.in);
+            cudaStreamSynchronize(cs.out);
+        }
+        return err;
+    };
 
     const size_t tok = (size_t)pr.N * pr.d;  // elements of one head of Q, K, V or O
     const size_t wsz = (size_t)pr.d * pr.d;  // elements of one head's weight matrix
@@ -89,59 +106,60 @@ veda_status forward_host_impl(const veda_problem* p, const Problem& pr, const ui
             pc.H = hc;
             pc.tile_shapes = p->tile_shapes + 3 * h0;
             Problem sub;
-            if ((st = make_problem(&pc, true, &sub))) return st;
+            if ((st = make_problem(&pc, true, &sub))) return fail_joined(st);
             const size_t off = ((size_t)b * pr.H + h0) * tok;
             const size_t bytes = (size_t)hc * tok * sizeof(uint16_t);
             // in: this chunk's Q, K, V (and weights, once per head)
             if ((st = cuda_check(cudaMemcpyAsync(dQ + off, hQ + off, bytes, cudaMemcpyHostToDevice,
                                                  cs.in), "Q copy in")))
-                return st;
+                return fail_joined(st);
             if ((st = cuda_check(cudaMemcpyAsync(dK + off, hK + off, bytes, cudaMemcpyHostToDevice,
                                                  cs.in), "K copy in")))
-                return st;
+                return fail_joined(st);
             if ((st = cuda_check(cudaMemcpyAsync(dV + off, hV + off, bytes, cudaMemcpyHostToDevice,
                                                  cs.in), "V copy in")))
-                return st;
+                return fail_joined(st);
             if (b == 0) {
                 const size_t wb = (size_t)hc * wsz * sizeof(float);
                 if ((st = cuda_check(cudaMemcpyAsync(dWq + h0 * wsz, hWq + h0 * wsz, wb,
                                                      cudaMemcpyHostToDevice, cs.in), "Wq copy in")))
-                    return st;
+                    return fail_joined(st);
                 if ((st = cuda_check(cudaMemcpyAsync(dWk + h0 * wsz, hWk + h0 * wsz, wb,
                                                      cudaMemcpyHostToDevice, cs.in), "Wk copy in")))
-                    return st;
+                    return fail_joined(st);
             }
             cudaEvent_t landed, computed;
-            if ((st = events.make(&landed)) || (st = events.make(&computed))) return st;
-            if ((st = cuda_check(cudaEventRecord(landed, cs.in), "event record"))) return st;
+            if ((st = events.make(&landed)) || (st = events.make(&computed))) return fail_joined(st);
+            if ((st = cuda_check(cudaEventRecord(landed, cs.in), "event record"))) return fail_joined(st);
             // compute: the whole layer on this chunk's heads
-            if ((st = cuda_check(cudaStreamWaitEvent(s, landed, 0), "stream wait"))) return st;
+            if ((st = cuda_check(cudaStreamWaitEvent(s, landed, 0), "stream wait"))) return fail_joined(st);
             float* lse_c = dlse ? dlse + ((size_t)b * pr.H + h0) * pr.N : nullptr;
             if ((st = forward_impl(sub, dQ + off, dK + off, dV + off, dWq + h0 * wsz,
                                    dWk + h0 * wsz, dO + off, lse_c, nullptr, nullptr, ws, s)))
-                return st;
-            if ((st = cuda_check(cudaEventRecord(computed, s), "event record"))) return st;
+                return fail_joined(st);
+            if ((st = cuda_check(cudaEventRecord(computed, s), "event record"))) return fail_joined(st);
             // out: this chunk's O (and lse)
             if ((st = cuda_check(cudaStreamWaitEvent(cs.out, computed, 0), "stream wait")))
-                return st;
+                return fail_joined(st);
             if ((st = cuda_check(cudaMemcpyAsync(hO + off, dO + off, bytes, cudaMemcpyDeviceToHost,
                                                  cs.out), "O copy out")))
-                return st;
+                return fail_joined(st);
             if (hlse != nullptr) {
                 const size_t lo = ((size_t)b * pr.H + h0) * pr.N;
                 if ((st = cuda_check(cudaMemcpyAsync(hlse + lo, dlse + lo,
                                                      (size_t)hc * pr.N * sizeof(float),
                                                      cudaMemcpyDeviceToHost, cs.out),
                                      "lse copy out")))
-                    return st;
+                    return fail_joined(st);
             }
         }
     }
     // the caller's stream completes only after the last copy out
     cudaEvent_t done;
-    if ((st = events.make(&done))) return st;
-    if ((st = cuda_check(cudaEventRecord(done, cs.out), "event record"))) return st;
-    return cuda_check(cudaStreamWaitEvent(s, done, 0), "stream wait");
+    if ((st = events.make(&done))) return fail_joined(st);
+    if ((st = cuda_check(cudaEventRecord(done, cs.out), "event record"))) return fail_joined(st);
+    if ((st = cuda_check(cudaStreamWaitEvent(s, done, 0), "stream wait"))) return fail_joined(st);
+    return VEDA_OK;
 }
 
 }  // namespace veda

@@ -21,6 +21,9 @@
 //   * every call shares the one array, which keeps the last call's contents:
 //     calls whose work overlaps on the GPU (other streams, other host threads)
 //     race on it; the status word is cleared by each call;
+//   * the device status word (VEDA_ERR_TIMEOUT when a bounded wait of the
+//     score kernel gave up) lives in the array too: veda_noalloc_get_status
+//     reads it back for the current device;
 //   * nothing here calls cudaMalloc, cudaFree or any allocating routine.
 #include <mutex>
 #include <string>
@@ -95,6 +98,18 @@ veda_status veda_tile_score_noalloc(const veda_problem* p, const float* statsQ,
     if ((st = veda::launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
     if ((st = veda::launch_project(pr, statsK, Wk, kt, 1, s))) return st;
     return veda::launch_score(pr, qt, kt, S, reinterpret_cast<int*>(base), s);
+}
+
+veda_status veda_noalloc_get_status(veda_stream_t stream, int32_t* device_status) {
+    if (device_status == nullptr) return veda::fail(VEDA_ERR_INVALID_ARG, "device_status is NULL");
+    void* scratch = nullptr;
+    veda_status st;
+    if ((st = scratch_for_current_device(&scratch)) != VEDA_OK) return st;
+    if ((st = veda::cuda_check(cudaStreamSynchronize((cudaStream_t)stream), "stream sync")))
+        return st;
+    return veda::cuda_check(
+        cudaMemcpy(device_status, scratch, sizeof(int32_t), cudaMemcpyDeviceToHost),
+        "status read");
 }
 
 }  // extern "C"

@@ -329,33 +329,6 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
     return d;
 }
 
-// 2^x for a pair of floats on the FMA and integer pipes (no MUFU):
-// Cody-Waite style split x = n + f, n = round(x) taken from the low mantissa
-// bits of x + 1.5*2^23 (exact in fp32), f = x - n in [-1/2, 1/2]; 2^f by a
-// cubic minimax fit (max relative error 7.5e-5, see fit_exp2_poly.py); 2^n is
-// added to the exponent field.  Inputs are clamped to >= -125 so every result
-// is a normal float; inputs above +126 are not supported (the softmax feeds
-// values <= 8).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-    constexpr float c0 = 9.999280572e-01f, c1 = 6.932609677e-01f, c2 = 2.426111251e-01f,
-                    c3 = 5.517166853e-02f;
-    float x0, x1;
-    f32x2_unpack(x, x0, x1);
-    x = f32x2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t t = f32x2_add(x, f32x2_pack(kMagic, kMagic));
-    const uint64_t n = f32x2_add(t, f32x2_pack(-kMagic, -kMagic));
-    const uint64_t f = f32x2_fma(n, f32x2_pack(-1.f, -1.f), x);
-    uint64_t q = f32x2_fma(f32x2_pack(c3, c3), f, f32x2_pack(c2, c2));
-    q = f32x2_fma(q, f, f32x2_pack(c1, c1));
-    q = f32x2_fma(q, f, f32x2_pack(c0, c0));
-    float t0, t1, q0, q1;
-    f32x2_unpack(t, t0, t1);
-    f32x2_unpack(q, q0, q1);
-    return f32x2_pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
-                      __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
-}
-
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

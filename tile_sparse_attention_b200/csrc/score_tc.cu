@@ -20,7 +20,8 @@
 //     (M = N = 128, K = 8) per K block;
 //   * all four warps read the accumulator back (thread = row) and store S.
 // Waits are bounded (VEDA_ERR_TIMEOUT in the status word, then a bounded drain
-// of the copies and products in flight before tensor memory is freed).
+// of the copies and products in flight before tensor memory is freed; S is not
+// written by a CTA that gave up).
 #include "internal.h"
 #include "kernel_common.cuh"
 #include "ptx.cuh"
@@ -45,6 +46,7 @@ struct __align__(64) ScoreParams {
     int* status;
     int nT, kblocks;
     unsigned long long wait_limit_ns;
+    int withhold_fill;  // failure-detection test only: the first K block is never loaded
 };
 
 __global__ void __launch_bounds__(kScoreThreads, 1)
@@ -92,6 +94,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         for (int kb = 0; kb < KB; ++kb) {
             const int st = kb % kStages, n = kb / kStages;
             if (n > 0 && !wait_bar(&empty[st], (n - 1) & 1, p, abort_flag)) break;
+            if (p.withhold_fill && kb == 0) {
+                // test hook: stage 0's first fill never happens, so the issuer's
+                // wait on it runs out (and stage 0 is never refilled)
+                issued = 1;
+                continue;
+            }
             uint8_t* a = smem + st * kStageBytes;
             mbar_arrive_expect_tx(&full[st], kStageBytes);
             tma_load_2d(a, &p.mapA, &full[st], kb * 32, rowA);
@@ -99,7 +107,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             issued = kb + 1;
         }
         for (int st = 0; st < kStages; ++st)  // drain: the last fill of every stage
-            if (st < issued) drain_bar(&full[st], ((issued - 1 - st) / kStages) & 1, p);
+            if (st < issued && !(p.withhold_fill && st == 0))
+                drain_bar(&full[st], ((issued - 1 - st) / kStages) & 1, p);
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------- MMA issuer
         const uint32_t base = smem_addr(smem);
@@ -127,7 +136,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     // -------------------------------------------------------------- epilogue
     int got = 0;
-    if (lane == 0) got = wait_bar(done, 0, p, abort_flag) ? 1 : 0;
+    // after an abort the accumulator is incomplete: S is not written
+    if (lane == 0) got = (wait_bar(done, 0, p, abort_flag) && !*abort_flag) ? 1 : 0;
     got = __shfl_sync(0xffffffffu, got, 0);
     __syncwarp();
     if (got) {
@@ -182,6 +192,8 @@ veda_status launch_score(const Problem& pr, const float* qext, const float* kext
     prm.nT = pr.nT;
     prm.kblocks = kx / 32;
     prm.wait_limit_ns = wait_limit_ns();
+    // Test hook for the bounded waits (nothing in normal use sets the variable).
+    prm.withhold_fill = getenv("VEDA_TEST_WITHHOLD_ARRIVE") != nullptr ? 1 : 0;
     cudaError_t err = cudaFuncSetAttribute(score_tc_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return cuda_check(err, "score smem attribute");

@@ -51,10 +51,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kSoftmaxWarp0 = 4;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-#ifndef VEDA_POLY_PAIRS
-#define VEDA_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = VEDA_POLY_PAIRS;  // of every 8 exp2 pairs, on the FMA pipe
 
 struct __align__(64) AttnParams {
     CUtensorMap tmQ[kMaxShapes];
@@ -383,10 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_use = need ? m_new : m_run;
                 alpha = need ? fast_exp2(m_run - m_new) : 1.f;
             }
-            // p = 2^(s*c2 - m): packed fp32x2 scale-and-shift; kPolyPairs of
-            // every 8 element pairs take the FMA-pipe exp2, the others MUFU
-            // ex2 (the two units then share the load); four independent packed
-            // partial sums
+            // p = 2^(s*c2 - m): packed fp32x2 scale-and-shift, MUFU ex2, four
+            // independent packed partial sums
             uint32_t pk[BT / 2];
             const uint64_t c2x2 = f32x2_pack(c2, c2);
             const uint64_t negm = f32x2_pack(-m_use, -m_use);
@@ -395,15 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < BT; e += 2) {
                 const uint64_t x = f32x2_fma(
                     f32x2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2x2, negm);
-                float p0, p1;
-                if (((e >> 1) & 7) < kPolyPairs) {
-                    f32x2_unpack(exp2_poly_x2(x), p0, p1);
-                } else {
-                    float x0, x1;
-                    f32x2_unpack(x, x0, x1);
-                    p0 = fast_exp2(x0);
-                    p1 = fast_exp2(x1);
-                }
+                float x0, x1;
+                f32x2_unpack(x, x0, x1);
+                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
                 acc[(e >> 1) & 3] = f32x2_add(acc[(e >> 1) & 3], f32x2_pack(p0, p1));
                 pk[e / 2] = pack_bf16x2(p0, p1);
             }
