@@ -1,15 +1,19 @@
-"""Barrier protocols of the two attention kernels, checked by random interleaving.
+"""Barrier protocols of the three attention kernels, checked by random interleaving.
 
 The tile-skipping attention kernels (sparse_attn.cu: one CTA per query tile;
 sparse_attn_persistent.cu: persistent CTAs looping over query tiles with one
-key-tile stream) hand work between a TMA producer thread, one tcgen05-issuing
-thread and four softmax warps through mbarriers waited on by phase parity.
-This module models those protocols -- the roles, the barriers and their arrival
-counts, a tensor pipe that executes in issue order, copies that land in any
-order -- and runs them under many random interleavings, checking that
+key-tile stream; sparse_attn_dual.cu: one query tile per CTA, two softmax
+groups on alternate 64-key chunks) hand work between TMA producer threads, one
+tcgen05-issuing thread and softmax warps through mbarriers waited on by phase
+parity.  This module models those protocols -- the roles, the barriers and
+their arrival counts, a tensor pipe that executes in issue order, copies that
+land in any order -- and runs them under many random interleavings, checking
+that
 
 * every role finishes (no deadlock);
-* no wait trails its barrier by two completions (the parity would alias);
+* every wait for completion c of a barrier happens while completion c - 1
+  has occurred and c + 1 has not (a parity wait is exact only then: two
+  phases behind it waits for ever, one phase ahead it passes at once);
 * every product reads what it should: the ring stage holds K_g / V_g, the
   S/P buffer holds S_g / P_g, tensor memory holds Q of the right query tile;
 * a query tile's output accumulator is read by the epilogue only after its
@@ -41,8 +45,12 @@ class Bar:
 
 
 def passed(bar, c):
-    """A wait for completion number c of `bar` (the kernels wait on parity c & 1)."""
+    """A wait for completion number c of `bar`.  The kernels wait on parity c & 1,
+    which is right only while completion c - 1 has happened and c + 1 has not:
+    a waiter two phases behind would wait for ever, and one that starts while
+    completion c - 1 is still pending would pass at once."""
     assert bar.done <= c + 1, f"wait for completion {c} trails the barrier ({bar.done} done)"
+    assert bar.done >= c, f"wait for completion {c} runs ahead of the barrier ({bar.done} done)"
     return bar.done >= c + 1
 
 
@@ -282,6 +290,159 @@ def model_persistent(n_tiles, k, NS, seed, p_rescale=0.3):
             st["O_read"][w] = n
 
     run([producer(), issuer()] + [softmax(w) for w in range(4)], tma, tc, rnd)
+
+
+# ------------------------------------------------------------------ two softmax groups
+def model_dual(k, seed, p_rescale=0.3, release_wait=True, q_gate=True, pv_wait=True,
+               free_wait=True, NS=6):
+    """sparse_attn_dual.cu: one query tile; its selected key tiles are processed
+    in 64-key chunks n = 0..2k-1 from one ring (two producers taking alternate
+    key tiles, each with its own 3 stages; Q staged in the last stage, gated by
+    q_tmem); three S/P buffers (chunk n in buffer n % 3); softmax group
+    g = n % 2 takes alternate chunks and accumulates its own O_g.  One thread
+    issues S(0..2), then per chunk: wait P(n), O_g += P(n) V (commits: stage
+    release, pv_done[g], and o_done[g] after the group's last), then
+    S(n + 3) = Q K^T into the buffer P(n) V read.  A group rescales O_g only
+    after pv_done[g] reports its previous P V, and reads O_g (both groups'
+    accumulators, after a barrier of the eight warps) after o_done[g].
+    free_wait=False plants S(n + 3) ahead of P(n) V in the issue order."""
+    rnd = random.Random(seed)
+    chunks = 2 * k
+    q_full, q_tmem = Bar(1), Bar(8)
+    k_full = [Bar(1) for _ in range(NS)]
+    v_full = [Bar(1) for _ in range(NS)]
+    kv_empty = [Bar(1) for _ in range(NS)]
+    s_full = [Bar(1) for _ in range(3)]
+    p_full = [Bar(4) for _ in range(3)]
+    pv_done = [Bar(1), Bar(1)]
+    o_done = [Bar(1), Bar(1)]
+    tma, tc = [], []
+    st = {"K": [None] * NS, "V": [None] * NS, "Qt": [False] * 8, "S": [None] * 3,
+          "P": [[None] * 4 for _ in range(3)], "Pread": [-1] * 3, "O": [0, 0],
+          "read": [False, False]}
+    mine = [False, False]
+    R = NS // 2
+
+    def stage(n):
+        j, hh = n >> 1, n & 1
+        m = 2 * (j >> 1) + hh
+        return R * (j & 1) + m % R, m // R
+
+    def q_loader():
+        def q_landed():
+            st["K"][NS - 1] = "Q"
+            q_full.arrive()
+        tma.append(q_landed)
+        yield lambda: passed(q_full, 0)
+
+    def producer(par):
+        for j in range(par, k, 2):
+            for hh in range(2):
+                n = 2 * j + hh
+                s, u = stage(n)
+                if u > 0 and release_wait:
+                    yield lambda: passed(kv_empty[s], u - 1)
+                elif u == 0 and s == NS - 1 and q_gate:
+                    yield lambda: passed(q_tmem, 0)
+
+                def kl(s=s, n=n):
+                    st["K"][s] = n
+                    k_full[s].arrive()
+
+                def vl(s=s, n=n):
+                    st["V"][s] = n
+                    v_full[s].arrive()
+                tma.append(kl)
+                tma.append(vl)
+
+    def issue_qk(n):
+        s, u = stage(n)
+        b = n % 3
+        yield lambda: passed(k_full[s], u)
+
+        def op(n=n, s=s, b=b):
+            assert st["K"][s] == n, "Q K^T read a ring stage that no longer holds its K half"
+            assert all(st["Qt"]), "Q K^T before Q reached tensor memory"
+            assert n < 3 or st["Pread"][b] == n - 3, \
+                "S overwrote a P buffer before its P V product read it"
+            st["S"][b] = n
+        tc.append(op)
+        tc.append(s_full[b].arrive)
+
+    def issuer():
+        yield lambda: passed(q_tmem, 0)
+        for n in range(min(3, chunks)):
+            yield from issue_qk(n)
+        for n in range(chunks):
+            s, u = stage(n)
+            b, g = n % 3, n % 2
+            yield lambda: passed(p_full[b], n // 3)
+            yield lambda: passed(v_full[s], u)
+            if not free_wait and n + 3 < chunks:  # planted: S(n + 3) ahead of P(n) V
+                yield from issue_qk(n + 3)
+
+            def op(n=n, s=s, b=b, g=g):
+                assert st["V"][s] == n, "P V read a ring stage that no longer holds its V half"
+                assert all(st["P"][b][w] == n for w in range(4)), "P V read a stale P buffer"
+                assert st["S"][b] == n, "the P buffer was overwritten before P V read it"
+                assert st["O"][g] == n // 2
+                assert not st["read"][g], "P V after the epilogue read O"
+                st["Pread"][b] = n
+                st["O"][g] += 1
+            tc.append(op)
+            tc.append(kv_empty[s].arrive)
+            tc.append(pv_done[g].arrive)
+            if n + 2 >= chunks:
+                tc.append(o_done[g].arrive)
+            if free_wait and n + 3 < chunks:
+                yield from issue_qk(n + 3)
+
+    def softmax(g, w):
+        yield lambda: passed(q_full, 0)
+        assert st["K"][NS - 1] == "Q", "the Q staging was overwritten before the copy"
+        st["Qt"][4 * g + w] = True
+        q_tmem.arrive()
+        i = 0
+        for n in range(g, chunks, 2):
+            b = n % 3
+            yield lambda: passed(s_full[b], n // 3)
+            assert st["S"][b] == n, "the softmax read a stale S buffer"
+            if i > 0 and rnd.random() < p_rescale:  # O_g rescale
+                if pv_wait:
+                    yield lambda: passed(pv_done[g], i - 1)
+                assert st["O"][g] == i, "O rescaled before the group's previous P V landed"
+            st["P"][b][w] = n
+            p_full[b].arrive()
+            i += 1
+        yield lambda: passed(o_done[g], 0)
+        assert st["O"][g] == i, "the epilogue read O before the group's last P V product"
+        # the merge reads both accumulators, after both groups passed this point
+        # (a barrier over the eight softmax warps)
+        mine[g] = True
+        yield lambda: all(mine)
+        assert st["O"] == [(chunks + 1) // 2, chunks // 2]
+        st["read"][g] = True
+
+    run([q_loader(), producer(0), producer(1), issuer()]
+        + [softmax(g, w) for g in range(2) for w in range(4)], tma, tc, rnd)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 7])
+def test_dual_protocol(k):
+    for seed in range(30):
+        model_dual(k, seed)
+
+
+def test_dual_planted_mistakes_are_caught():
+    for kw in (dict(release_wait=False), dict(q_gate=False), dict(pv_wait=False),
+               dict(free_wait=False)):
+        caught = 0
+        for seed in range(40):
+            try:
+                model_dual(5, seed, **kw)
+            except AssertionError:
+                caught += 1
+        assert caught > 0, kw
 
 
 @pytest.mark.parametrize("NS", [2, 3, 4])

@@ -80,11 +80,23 @@ veda_status launch_sparse_attn_persistent(const Problem& pr, const uint16_t* Q,
                                           const int32_t* idx, int k, uint16_t* O, float* lse,
                                           int* status, cudaStream_t s);
 
+// One query tile per CTA, two softmax groups on alternate 64-key chunks
+// (sparse_attn_dual.cu): d = 128 and 128-token tiles, k >= kDualMinK.
+constexpr int kDualMinK = 8;
+bool dual_attn_supported(const Problem& pr);
+veda_status launch_sparse_attn_dual(const Problem& pr, const uint16_t* Q, const uint16_t* K,
+                                    const uint16_t* V, const int32_t* idx, int k, uint16_t* O,
+                                    float* lse, int* status, cudaStream_t s);
+
 // TMA descriptors (tensor_maps.cu): the 5-D tile view (d, Ws, Hs, T, B*H) of a
 // [B,H,N,d] bf16 tensor with a (64, p_w, p_h, p_t, 1) box, and a 2-D row view
 // of an fp32 [rows][cols] matrix with a (32, 128) box; both 128-byte swizzled.
 veda_status encode_tile_map(CUtensorMap* map, const void* base, const Problem& pr,
                             const int* shape);
+// The same tile view for d = 128 with both 64-channel chunks in one box:
+// dims (64, Ws, Hs, T*B*H, 2), box (64, p_w, p_h, p_t, 2) -> two 128-row planes.
+veda_status encode_tile_map_2c(CUtensorMap* map, const void* base, const Problem& pr,
+                               const int* shape);
 veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows, int cols);
 // Time limit of a device wait (VEDA_WAIT_LIMIT_MS, default 10 s).
 unsigned long long wait_limit_ns();

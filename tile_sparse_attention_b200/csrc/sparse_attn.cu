@@ -1,6 +1,8 @@
 // sparse_attn.cu -- tile-skipping flash attention for sm_100a (tcgen05 + TMEM + TMA),
-// one CTA per query tile (used for k > kPersistentMaxK; shorter key lists go to
-// the persistent kernel in sparse_attn_persistent.cu).
+// one CTA per query tile.  Used for k > kPersistentMaxK when the head dimension
+// or the tile size is 64 (shorter key lists go to the persistent kernel in
+// sparse_attn_persistent.cu); d = 128 with 128-token tiles goes to the
+// two-group kernel in sparse_attn_dual.cu.  launch_sparse_attn below picks.
 //
 // "Veda: Scalable Video Diffusion via Distilled Sparse Attention" (project
 // page): "Attention Structure Distillation", Execution (the tile mask is
@@ -259,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
+        if (elect_one()) {
             const uint32_t tS = tbase + C::kTmemS;
             const uint32_t tQ = tbase + C::kTmemQ;
             const uint32_t tO = tbase + C::kTmemO;
@@ -506,9 +508,15 @@ veda_status launch_cfg(const AttnParams& prm, const Problem& pr, cudaStream_t s)
 veda_status launch_sparse_attn(const Problem& pr, const uint16_t* Q, const uint16_t* K,
                                const uint16_t* V, const int32_t* idx, int k, uint16_t* O,
                                float* lse, int* status, cudaStream_t s) {
-    // Short key lists: the per-CTA fixed cost (allocation, Q load, pipeline fill,
-    // epilogue) dominates, and the persistent kernel that carries its pipeline
-    // across query tiles is faster; long ones: this kernel's steady state is.
+    // d = 128 with 128-token tiles: two softmax groups per query tile on
+    // alternate 64-key chunks (two softmax warps share each SM sub-partition
+    // and feed the tensor core), except for very short key lists, where the
+    // persistent kernel's lower fixed cost per query tile wins (measured:
+    // k = 2 faster there, k = 12 even, k >= 30 8-11% slower)
+    if (dual_attn_supported(pr) && k >= kDualMinK)
+        return launch_sparse_attn_dual(pr, Q, K, V, idx, k, O, lse, status, s);
+    // other shapes: short key lists go to the persistent kernel that carries
+    // its pipeline across query tiles, long ones to this kernel
     if (k <= kPersistentMaxK)
         return launch_sparse_attn_persistent(pr, Q, K, V, idx, k, O, lse, status, s);
     AttnParams prm;
