@@ -309,8 +309,7 @@ def model_dual(k, seed, p_rescale=0.3, release_wait=True, q_gate=True, pv_wait=T
     rnd = random.Random(seed)
     chunks = 2 * k
     q_full, q_tmem = Bar(1), Bar(8)
-    k_full = [Bar(1) for _ in range(NS)]
-    v_full = [Bar(1) for _ in range(NS)]
+    kv_full = [Bar(1) for _ in range(NS)]  # K and V halves land on one barrier
     kv_empty = [Bar(1) for _ in range(NS)]
     s_full = [Bar(1) for _ in range(3)]
     p_full = [Bar(4) for _ in range(3)]
@@ -345,20 +344,17 @@ def model_dual(k, seed, p_rescale=0.3, release_wait=True, q_gate=True, pv_wait=T
                 elif u == 0 and s == NS - 1 and q_gate:
                     yield lambda: passed(q_tmem, 0)
 
-                def kl(s=s, n=n):
+                def kvl(s=s, n=n):
+                    # the barrier completes once both copies landed
                     st["K"][s] = n
-                    k_full[s].arrive()
-
-                def vl(s=s, n=n):
                     st["V"][s] = n
-                    v_full[s].arrive()
-                tma.append(kl)
-                tma.append(vl)
+                    kv_full[s].arrive()
+                tma.append(kvl)
 
     def issue_qk(n):
         s, u = stage(n)
         b = n % 3
-        yield lambda: passed(k_full[s], u)
+        yield lambda: passed(kv_full[s], u)
 
         def op(n=n, s=s, b=b):
             assert st["K"][s] == n, "Q K^T read a ring stage that no longer holds its K half"
@@ -376,8 +372,7 @@ def model_dual(k, seed, p_rescale=0.3, release_wait=True, q_gate=True, pv_wait=T
         for n in range(chunks):
             s, u = stage(n)
             b, g = n % 3, n % 2
-            yield lambda: passed(p_full[b], n // 3)
-            yield lambda: passed(v_full[s], u)
+            yield lambda: passed(p_full[b], n // 3)  # V landed with K (S(n) waited)
             if not free_wait and n + 3 < chunks:  # planted: S(n + 3) ahead of P(n) V
                 yield from issue_qk(n + 3)
 

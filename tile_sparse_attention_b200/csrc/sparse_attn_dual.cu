@@ -79,9 +79,9 @@ constexpr int kQChunk = 128 * 128;
 constexpr int kQBytes = 2 * kQChunk;
 constexpr int kQStage = kStages - 1;  // Q staged in the last stage (producer 1's third)
 constexpr int kOffBar = kStages * kStageBytes;
-// barriers: q_full, q_tmem, k_full[6], v_full[6], kv_empty[6], s_full[3],
+// barriers: q_full, q_tmem, kv_full[6], kv_empty[6], s_full[3],
 // p_full[3], pv_done[2], o_done[2], drain
-constexpr int kNumBars = 2 + 3 * kStages + 3 + 3 + 2 + 2 + 1;
+constexpr int kNumBars = 2 + 2 * kStages + 3 + 3 + 2 + 2 + 1;
 constexpr int kOffML = kOffBar + 512;          // per-row (max, sum) of both groups
 constexpr int kOffMisc = kOffML + 2 * 128 * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -116,8 +116,7 @@ struct __align__(64) DualParams {
 struct Bars {
     uint64_t* q_full;
     uint64_t* q_tmem;
-    uint64_t* k_full;
-    uint64_t* v_full;
+    uint64_t* kv_full;
     uint64_t* kv_empty;
     uint64_t* s_full;
     uint64_t* p_full;
@@ -146,7 +145,7 @@ __device__ __forceinline__ void issue_all(const DualParams& p, const Bars& bars,
     auto issue_qk = [&](int n) -> bool {
         int st, u;
         chunk_stage(n, st, u);
-        if (!wait_bar(&bars.k_full[st], u & 1, p, abort_flag)) return false;
+        if (!wait_bar(&bars.kv_full[st], u & 1, p, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kaddr = ring + st * kStageBytes;
         const uint32_t dS = tbase + kTmemS + 64 * (n % 3);
@@ -165,9 +164,8 @@ __device__ __forceinline__ void issue_all(const DualParams& p, const Bars& bars,
         const int b = n % 3, g = n & 1;
         int st, u;
         chunk_stage(n, st, u);
-        if (!wait_bar(&bars.p_full[b], (n / 3) & 1, p, abort_flag) ||
-            !wait_bar(&bars.v_full[st], u & 1, p, abort_flag))
-            break;
+        // the V half landed with the K half (one barrier), whose wait S(n) passed
+        if (!wait_bar(&bars.p_full[b], (n / 3) & 1, p, abort_flag)) break;
         tc_fence_after();
         // O_g += P(n) V: A = P(n) (bf16 pairs over S buffer b), B = the V half
         // (MN-major: 64-channel planes 8 KB apart, 16 keys per 2 KB)
@@ -193,7 +191,8 @@ __device__ __forceinline__ void issue_all(const DualParams& p, const Bars& bars,
 //   q_tmem              all eight softmax warps wrote their half of Q into
 //                       tensor memory: once; also gates the first fill of the
 //                       Q staging stage
-//   k_full/v_full[st]   use u of stage st has landed: parity u & 1
+//   kv_full[st]         use u of stage st (K and V halves) has landed:
+//                       parity u & 1
 //   kv_empty[st]        the P V of use u is done (one commit): parity u & 1
 //   s_full[b], p_full[b]  chunk n is use n div 3 of buffer b = n mod 3:
 //                       parity (n div 3) & 1
@@ -221,9 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     Bars bars;
     bars.q_full = bar_base;
     bars.q_tmem = bar_base + 1;
-    bars.k_full = bar_base + 2;
-    bars.v_full = bars.k_full + kStages;
-    bars.kv_empty = bars.v_full + kStages;
+    bars.kv_full = bar_base + 2;
+    bars.kv_empty = bars.kv_full + kStages;
     bars.s_full = bars.kv_empty + kStages;
     bars.p_full = bars.s_full + 3;
     bars.pv_done = bars.p_full + 3;
@@ -247,8 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bars.q_full, 1);
         mbar_init(bars.q_tmem, 8);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&bars.k_full[s], 1);
-            mbar_init(&bars.v_full[s], 1);
+            mbar_init(&bars.kv_full[s], 1);
             mbar_init(&bars.kv_empty[s], 1);
         }
         for (int b = 0; b < 3; ++b) {
@@ -326,11 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             good = wait_bar(bars.q_tmem, 0, p, abort_flag);
                         if (good) {
                             uint8_t* sk = smem + st * kStageBytes;
-                            mbar_arrive_expect_tx(&bars.k_full[st], kHalfBytes);
-                            tma_load_5d(sk, &p.tmK[slot], &bars.k_full[st], 0, x0 + hh * dx,
+                            mbar_arrive_expect_tx(&bars.kv_full[st], 2 * kHalfBytes);
+                            tma_load_5d(sk, &p.tmK[slot], &bars.kv_full[st], 0, x0 + hh * dx,
                                         y0 + hh * dy, t0 + hh * dt, 0);
-                            mbar_arrive_expect_tx(&bars.v_full[st], kHalfBytes);
-                            tma_load_5d(sk + kHalfBytes, &p.tmV[slot], &bars.v_full[st], 0,
+                            tma_load_5d(sk + kHalfBytes, &p.tmV[slot], &bars.kv_full[st], 0,
                                         x0 + hh * dx, y0 + hh * dy, t0 + hh * dt, 0);
                             fills = m + 1;
                         }
@@ -345,8 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int r = 0; r < kRing; ++r) {
                 if (r < fills) {
                     const uint32_t par = ((fills - 1 - r) / kRing) & 1;
-                    drain_bar(&bars.k_full[kRing * pr + r], par, p);
-                    drain_bar(&bars.v_full[kRing * pr + r], par, p);
+                    drain_bar(&bars.kv_full[kRing * pr + r], par, p);
                 }
             }
         }
@@ -421,7 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_new = fmaxf(m_run, m_tile);
                 need = m_new > m_run + kRescaleThreshold;
                 m_use = need ? m_new : m_run;
-                alpha = need ? fast_exp2(m_run - m_new) : 1.f;
+                alpha = 1.f;
+                // the MUFU is shared with the other group's exponentials on
+                // this sub-partition: only a rescale pays for this one
+                if (__any_sync(0xffffffffu, need) && need) alpha = fast_exp2(m_run - m_new);
             }
             // p = 2^(s*c2 - m): packed fp32x2 scale-and-shift, MUFU ex2, four
             // independent packed partial sums
