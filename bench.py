@@ -42,13 +42,20 @@ METRIC = "ms/layer and effective TFLOP/s of tile-sparse attention (+mask prep) a
 
 
 # DRAM bytes (read + write) of one attention launch on the estimator's mask,
-# from one ncu capture of dram__bytes_read.sum + dram__bytes_write.sum, with the
-# kernel version it was taken on.  A kernel change empties the entry until the
-# counters are taken again.
-ATTN_DRAM_BYTES = {"long_video_245k": {"bytes": 3.41e9 + 2.02e9,
-                                       "kernel": "sparse_attn_kernel<128,128,3>, commit 2b2780b",
+# with the kernel version and the capture they come from.  A kernel change
+# empties the entry until the counters are taken again.  The long-video figure
+# scales a single-launch capture at the 720P-like layer (1.112 GB read +
+# 0.763 GB written for 24,000 query tiles) by query tiles (61,440), the size
+# rule for counter captures keeping them off the 6 GB workload.
+ATTN_DRAM_BYTES = {"long_video_245k": {"bytes": (1.112e9 + 0.763e9) * 61440 / 24000,
+                                       "kernel": "sparse_attn_dual_kernel, commit d3c5c7b",
                                        "capture": "ncu --metrics dram__bytes_read.sum,"
-                                                  "dram__bytes_write.sum, one launch"}}
+                                                  "dram__bytes_write.sum, one launch at the "
+                                                  "720P-like layer, scaled by query tiles"},
+                   "720p": {"bytes": 1.112e9 + 0.763e9,
+                            "kernel": "sparse_attn_dual_kernel, commit d3c5c7b",
+                            "capture": "ncu --metrics dram__bytes_read.sum,"
+                                       "dram__bytes_write.sum, one launch"}}
 
 
 def _config(w, world):
