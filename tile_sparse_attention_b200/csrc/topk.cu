@@ -6,8 +6,10 @@
 // query tile produces the tile mask handed to the tile-skipping kernel.  Ties
 // go to the lower tile index; -0.0 and +0.0 tie.
 //
-// One warp per row.  The row is read with 16-byte loads (up to sixteen in flight
-// per lane) into shared memory.  The selection is exact and integer-valued:
+// One warp per row, in one of two kernels.  Rows of up to 2048 scores stay in
+// registers (topk_reg_kernel, described where it is defined).  Longer rows are
+// read with 16-byte loads (up to sixteen in flight per lane) into shared
+// memory (topk_kernel).  The selection is exact and integer-valued:
 //   1. Bucketing: every score goes to one of 256 buckets spread linearly over
 //      [row min, row max].  The bucket index is computed with correctly
 //      rounded fp32 operations from the score alone, so it is a
@@ -343,6 +345,332 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(const __grid_constant_
     }
 }
 
+// ---------------------------------------------------------------------------
+// Rows of up to 2048 scores: the row stays in registers.
+//
+// Lane l holds the float4 groups l, l + 32, ... (G of them), and the next row
+// is loaded into the same registers once the current one's bucket b* scores
+// have been gathered, so its loads land while this row's selection finishes.  The scores become 7-bit buckets,
+//   bucket(x) = floor(127 * sat(fl(fl(x - min) * inv))),  inv = 1 / (max - min),
+// a non-decreasing function of x in which equal scores (-0.0 and +0.0
+// included) share a bucket; `sat` clamps to [0, 1] and sends NaN to 0, so the
+// padding of a short last group (NaN) lands in bucket 0 and never counts.  Four
+// buckets are packed per register, each byte with its top bit set, so that
+// byte-wise `b >= P` is the top bit of the byte after subtracting P (no byte
+// borrows).  Then, with no shared-memory histogram:
+//   1. a binary search over the 128 buckets, each probe a byte-parallel count
+//      reduced over the warp, gives the bucket b* of the k-th largest score and
+//      the number of scores above it;
+//   2. the scores of bucket b* (a handful for smooth rows) are gathered from
+//      the registers and their exact threshold found as in the kernel above (pairwise ranks for up to 32,
+//      an 8-bit radix select otherwise, or over the whole row if more than
+//      kCandCap share the bucket); the chosen ones of b* are marked in a bitmap;
+//   3. the selected bytes of every packed word (buckets above b*, plus the
+//      bitmap) give per-lane counts, whose prefix over the warp comes from four
+//      counts per 32-bit word in one scan, and the index list is written already
+//      ascending.
+
+constexpr int kRegWarps = 4;
+constexpr int kRegMaxG = 16;                 // rows of up to 128 * 16 = 2048 scores
+constexpr int kRegBitmapWords = 2048 / 32;   // one bit per score
+// per warp: histogram, candidate keys, candidate indices, bitmap, counter (16 B)
+constexpr int kRegWarpWords = kBins + 2 * kCandCap + kRegBitmapWords + 4;
+
+// Bit pattern of fl(2^23 + 127 t), rounded toward zero, for t = sat(fl(fl(x - mn) * inv)):
+// its low byte is floor(127 t), the bucket of x (0..127).
+__device__ __forceinline__ uint32_t bucket7_bits(float x, float mn, float inv) {
+    float d, t, r;
+    asm("sub.rn.f32 %0, %1, %2;" : "=f"(d) : "f"(x), "f"(mn));
+    asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(t) : "f"(d), "f"(inv));
+    asm("fma.rz.f32 %0, %1, 0f42FE0000, 0f4B000000;" : "=f"(r) : "f"(t));  // 127, 2^23
+    return __float_as_uint(r);
+}
+
+__device__ __forceinline__ uint32_t bucket7(float x, float mn, float inv) {
+    return bucket7_bits(x, mn, inv) & 0x7fu;
+}
+
+// Four buckets in one word, each byte 0x80 | bucket.
+__device__ __forceinline__ uint32_t pack_buckets(const float4& v, float mn, float inv) {
+    const uint32_t lo = __byte_perm(bucket7_bits(v.x, mn, inv), bucket7_bits(v.y, mn, inv), 0x0040);
+    const uint32_t hi = __byte_perm(bucket7_bits(v.z, mn, inv), bucket7_bits(v.w, mn, inv), 0x0040);
+    return __byte_perm(lo, hi, 0x5410) | 0x80808080u;
+}
+
+// Group g (scores 4g .. 4g+3) of a row; scores beyond nT read as NaN.
+template <bool ALIGNED>
+__device__ __forceinline__ float4 load_group(const float* srow, int g, int nT) {
+    const float qnan = __int_as_float(0x7fc00000);
+    if (ALIGNED) {
+        if (4 * g < nT) return __ldg(reinterpret_cast<const float4*>(srow) + g);
+        return make_float4(qnan, qnan, qnan, qnan);
+    }
+    const int j = 4 * g;
+    float4 v;
+    v.x = j < nT ? __ldg(srow + j) : qnan;
+    v.y = j + 1 < nT ? __ldg(srow + j + 1) : qnan;
+    v.z = j + 2 < nT ? __ldg(srow + j + 2) : qnan;
+    v.w = j + 3 < nT ? __ldg(srow + j + 3) : qnan;
+    return v;
+}
+
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));  // NaN inputs ignored
+    return r;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+template <int G, bool ALIGNED>
+__global__ void __launch_bounds__(kRegWarps * 32, G >= 12 ? 4 : G >= 5 ? 5 : 6)
+    topk_reg_kernel(const __grid_constant__ TopkParams p) {
+    __shared__ __align__(16) uint32_t smem_u[kRegWarps * kRegWarpWords];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* hist = smem_u + warp * kRegWarpWords;
+    uint32_t* ck = hist + kBins;
+    int32_t* ci = reinterpret_cast<int32_t*>(ck + kCandCap);
+    uint32_t* bm = reinterpret_cast<uint32_t*>(ci + kCandCap);
+    uint32_t* ncand = bm + kRegBitmapWords;
+    const unsigned full = 0xffffffffu;
+    const int nT = p.nT, k = p.k;
+    const long long stride = (long long)gridDim.x * kRegWarps;
+    long long row = (long long)blockIdx.x * kRegWarps + warp;
+
+    float4 v[G];
+    if (row < p.rows) {
+#pragma unroll
+        for (int u = 0; u < G; ++u) v[u] = load_group<ALIGNED>(p.S + row * nT, 32 * u + lane, nT);
+    }
+    for (; row < p.rows; row += stride) {
+        const float* srow = p.S + row * nT;
+        // ---- row min and max (the NaN padding is ignored)
+        float mn0 = INFINITY, mn1 = INFINITY, mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < G; ++u) {
+            mn0 = min3f(mn0, v[u].x, v[u].y);
+            mn1 = min3f(mn1, v[u].z, v[u].w);
+            mx0 = max3f(mx0, v[u].x, v[u].y);
+            mx1 = max3f(mx1, v[u].z, v[u].w);
+        }
+        float mn = fminf(mn0, mn1), mx = fmaxf(mx0, mx1);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(full, mn, off));
+            mx = fmaxf(mx, __shfl_xor_sync(full, mx, off));
+        }
+        // a zero or non-finite range puts every score in bucket 0 (still exact)
+        const float range = __fsub_rn(mx, mn);
+        const float inv = (range > 0.f && range <= FLT_MAX) ? fminf(__frcp_rn(range), FLT_MAX) : 0.f;
+        uint32_t pk[G];
+#pragma unroll
+        for (int u = 0; u < G; ++u) pk[u] = pack_buckets(v[u], mn, inv);
+        for (int w = lane; w < kRegBitmapWords; w += 32) bm[w] = 0u;
+        if (lane == 0) *ncand = 0u;
+
+        // ---- 1. bucket b* of the k-th largest score: count(bucket >= lo) >= k > count(bucket >= hi)
+        uint32_t lo = 0, hi = 128, above = 0;
+#pragma unroll 1
+        for (int it = 0; it < 7; ++it) {
+            const uint32_t mid = (lo + hi) >> 1;
+            const uint32_t T = mid * 0x01010101u;
+            uint32_t acc[3] = {0u, 0u, 0u};  // three independent chains; bytes stay <= G
+#pragma unroll
+            for (int u = 0; u < G; ++u) acc[u % 3] += ((pk[u] - T) & 0x80808080u) >> 7;
+            const uint32_t a = acc[0] + acc[1] + acc[2];
+            const uint32_t c = __reduce_add_sync(full, (a * 0x01010101u) >> 24);
+            if (c >= (uint32_t)k) {
+                lo = mid;
+            } else {
+                hi = mid;
+                above = c;
+            }
+        }
+        const uint32_t bstar = lo;
+        int kr = k - (int)above;  // rank of the k-th largest score within bucket b*
+        __syncwarp();
+
+        // ---- 2. the scores of bucket b*, taken from the registers
+        const uint32_t Bs = bstar * 0x01010101u;
+#pragma unroll
+        for (int u = 0; u < G; ++u) {
+            const uint32_t z = (pk[u] ^ Bs) & 0x7f7f7f7fu;
+            uint32_t eq = ~(z + 0x7f7f7f7fu) & 0x80808080u;
+            if (eq != 0u) {
+                const int j0 = 4 * (32 * u + lane);
+                do {
+                    const int e = (__ffs(eq) - 8) >> 3;
+                    eq &= eq - 1u;
+                    if (j0 + e < nT) {
+                        const float x = e == 0 ? v[u].x : e == 1 ? v[u].y : e == 2 ? v[u].z : v[u].w;
+                        const uint32_t pos = atomicAdd(ncand, 1u);
+                        if (pos < (uint32_t)kCandCap) {
+                            ck[pos] = order_key(x);
+                            ci[pos] = j0 + e;
+                        }
+                    }
+                } while (eq != 0u);
+            }
+        }
+        // ---- the next row's loads go out now and land during the rest of this one
+        {
+            const long long nrow = row + stride;
+            if (nrow < p.rows) {
+#pragma unroll
+                for (int u = 0; u < G; ++u) v[u] = load_group<ALIGNED>(p.S + nrow * nT, 32 * u + lane, nT);
+            }
+        }
+        __syncwarp();
+        const int c = (int)*ncand;  // >= kr
+        uint32_t thr;
+        if (c <= kCandCap) {
+            thr = candidate_threshold(ck, c, kr, hist, lane);
+        } else {
+            thr = radix_select(
+                [&](auto&& f) {
+                    for (int j = lane; j < nT; j += 32) {
+                        const float x = __ldg(srow + j);
+                        if (bucket7(x, mn, inv) == bstar) f(order_key(x));
+                    }
+                },
+                kr, hist, lane);
+        }
+        // kr is now the number of scores equal to the threshold that are kept
+        // (the lowest-index ones); mark the chosen scores of b* in the bitmap
+        if (c <= kCandCap) {
+            int neq = 0;
+            for (int j = lane; j < c; j += 32) neq += ck[j] == thr ? 1 : 0;
+            neq = __reduce_add_sync(full, neq);
+            for (int j = lane; j < c; j += 32) {
+                const uint32_t key = ck[j];
+                const int id = ci[j];
+                bool keep = key > thr;
+                if (key == thr) {
+                    if (neq == kr) {
+                        keep = true;
+                    } else {
+                        int r = 0;
+                        for (int m = 0; m < c; ++m) r += (ck[m] == thr && ci[m] < id) ? 1 : 0;
+                        keep = r < kr;
+                    }
+                }
+                if (keep) atomicOr(&bm[id >> 5], 1u << (id & 31));
+            }
+        } else {
+            int eq_seen = 0;
+            const unsigned lt = (1u << lane) - 1u;
+            for (int j0 = 0; j0 < nT; j0 += 32) {
+                const int j = j0 + lane;
+                bool gt = false, eq = false;
+                if (j < nT) {
+                    const float x = __ldg(srow + j);
+                    if (bucket7(x, mn, inv) == bstar) {
+                        const uint32_t key = order_key(x);
+                        gt = key > thr;
+                        eq = key == thr;
+                    }
+                }
+                const unsigned be = __ballot_sync(full, eq);
+                const bool keep = gt || (eq && eq_seen + __popc(be & lt) < kr);
+                eq_seen += __popc(be);
+                const unsigned bk = __ballot_sync(full, keep);
+                if (lane == 0) bm[j0 >> 5] = bk;
+            }
+        }
+        __syncwarp();
+
+        // ---- 3. selected bytes, their prefix over the warp, the ascending list and the mask
+        const uint32_t T = (bstar + 1u) * 0x01010101u;
+        constexpr int NS = (G + 3) / 4;
+        uint32_t sw[NS];
+#pragma unroll
+        for (int q = 0; q < NS; ++q) sw[q] = 0u;
+#pragma unroll
+        for (int u = 0; u < G; ++u) {
+            const int g = 32 * u + lane;
+            const uint32_t nib = (bm[g >> 3] >> (4 * (g & 7))) & 0xfu;  // chosen scores of b*
+            const uint32_t m = ((pk[u] - T) & 0x80808080u) | (((nib * 0x00204081u) & 0x01010101u) << 7);
+            pk[u] = m;
+            sw[u >> 2] |= (uint32_t)__popc(m) << (8 * (u & 3));
+        }
+        uint32_t excl[NS], tot[NS];
+#pragma unroll
+        for (int q = 0; q < NS; ++q) {
+            uint32_t incl = sw[q];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t t = __shfl_up_sync(full, incl, off);
+                if (lane >= off) incl += t;  // each byte <= 32 * 4: no carries between counts
+            }
+            excl[q] = incl - sw[q];
+            tot[q] = __shfl_sync(full, incl, 31);
+        }
+        int32_t* irow = p.idx + row * k;
+        int run = 0;
+#pragma unroll
+        for (int u = 0; u < G; ++u) {
+            const int g = 32 * u + lane;
+            int q = run + (int)((excl[u >> 2] >> (8 * (u & 3))) & 0xffu);
+            run += (int)((tot[u >> 2] >> (8 * (u & 3))) & 0xffu);
+            const uint32_t m = pk[u];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if ((m >> (8 * e + 7)) & 1u) {
+                    if (q < k) irow[q] = 4 * g + e;  // exactly k are selected
+                    ++q;
+                }
+        }
+        if (p.mask != nullptr) {
+            uint8_t* mrow = p.mask + row * nT;
+#pragma unroll
+            for (int u = 0; u < G; ++u) {
+                const int g = 32 * u + lane;
+                const uint32_t flags = (pk[u] >> 7) & 0x01010101u;
+                if (ALIGNED) {
+                    if (4 * g < nT) reinterpret_cast<uint32_t*>(mrow)[g] = flags;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (4 * g + e < nT) mrow[4 * g + e] = (uint8_t)((flags >> (8 * e)) & 1u);
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+template <int G, bool ALIGNED>
+veda_status launch_topk_reg(const TopkParams& prm, cudaStream_t s) {
+    static const int per_sm = [] {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, topk_reg_kernel<G, ALIGNED>,
+                                                          kRegWarps * 32, 0) != cudaSuccess || n < 1)
+            n = 1;
+        return n;
+    }();
+    const long long need = (prm.rows + kRegWarps - 1) / kRegWarps;
+    const long long cap = (long long)per_sm * sm_count();
+    const unsigned blocks = (unsigned)(need < cap ? need : cap);
+    topk_reg_kernel<G, ALIGNED><<<blocks, kRegWarps * 32, 0, s>>>(prm);
+    return cuda_check(cudaGetLastError(), "topk launch");
+}
+
+template <bool ALIGNED>
+veda_status launch_topk_reg_g(const TopkParams& prm, int g, cudaStream_t s) {
+    if (g <= 1) return launch_topk_reg<1, ALIGNED>(prm, s);
+    if (g <= 2) return launch_topk_reg<2, ALIGNED>(prm, s);
+    if (g <= 4) return launch_topk_reg<4, ALIGNED>(prm, s);
+    if (g <= 5) return launch_topk_reg<5, ALIGNED>(prm, s);
+    if (g <= 8) return launch_topk_reg<8, ALIGNED>(prm, s);
+    if (g <= 12) return launch_topk_reg<12, ALIGNED>(prm, s);
+    if (g <= 15) return launch_topk_reg<15, ALIGNED>(prm, s);
+    return launch_topk_reg<16, ALIGNED>(prm, s);
+}
+
 template <int W, int LOADS>
 veda_status launch_topk_w(const TopkParams& prm, cudaStream_t s) {
     const size_t smem = topk_warp_words(prm.nT) * sizeof(uint32_t) * W;
@@ -365,10 +693,14 @@ veda_status launch_topk(const Problem& pr, const float* S, uint8_t* mask, int32_
     prm.rows = (long long)pr.B * pr.H * pr.nT;
     prm.nT = pr.nT;
     prm.k = pr.k;
-    // four warps (rows) per block up to 4096 tiles (<= 74 KB of shared memory),
-    // one above (<= 66 KB at the 16384-tile limit); eight loads in flight per
-    // lane cover a row of up to 1024 scores in one round
-    if (pr.nT <= 1024) return launch_topk_w<4, 8>(prm, s);
+    // rows of up to 2048 scores: in registers, 128 scores per float4 group of
+    // every lane; longer rows: in shared memory, four warps (rows) per block
+    // up to 4096 tiles (<= 74 KB), one above (<= 66 KB at the 16384-tile limit)
+    if (pr.nT <= 128 * kRegMaxG) {
+        const int g = (pr.nT + 127) / 128;
+        return (pr.nT & 3) == 0 ? launch_topk_reg_g<true>(prm, g, s)
+                                : launch_topk_reg_g<false>(prm, g, s);
+    }
     if (pr.nT <= 4096) return launch_topk_w<4, 16>(prm, s);
     return launch_topk_w<1, 16>(prm, s);
 }
