@@ -13,7 +13,7 @@
 //     chunk's rows) by TMA into a 3-stage ring -- the same operands, in the
 //     same order, as the stand-alone score kernel, so every S value is
 //     bit-identical to it;
-//   * warp 5 owns 256 TMEM columns (two S chunk buffers); its lane 0 issues the
+//   * warp 5 owns 256 TMEM columns (two S chunk buffers); one elected lane issues the
 //     kind::tf32 MMAs of chunk c into buffer c mod 2;
 //   * warps 0..3 (thread = row) read their row of chunk c out of tensor memory,
 //     release the buffer, and fold the 128 scores into a running Top-k: a
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
+        if (elect_one()) {
             const uint32_t base = smem_addr(smem);
             bool ok = true;
             for (int t = 0; t < NC && ok; ++t) {

@@ -16,8 +16,8 @@
 //   * one CTA per 128 x 128 block of S of one head; 128 threads;
 //   * warp 0 lane 0 streams 32-wide K blocks of q^ and k^ (128 rows x 128 B,
 //     128-byte swizzle) by TMA into a 3-stage ring;
-//   * warp 1 allocates 128 TMEM columns; its lane 0 issues 4 tcgen05.mma
-//     (M = N = 128, K = 8) per K block;
+//   * warp 1 allocates 128 TMEM columns; one of its lanes, chosen by
+//     elect.sync, issues 4 tcgen05.mma (M = N = 128, K = 8) per K block;
 //   * all four warps read the accumulator back (thread = row) and store S.
 // Waits are bounded (VEDA_ERR_TIMEOUT in the status word, then a bounded drain
 // of the copies and products in flight before tensor memory is freed; S is not
@@ -109,28 +109,32 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         for (int st = 0; st < kStages; ++st)  // drain: the last fill of every stage
             if (st < issued && !(p.withhold_fill && st == 0))
                 drain_bar(&full[st], ((issued - 1 - st) / kStages) & 1, p);
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        const uint32_t base = smem_addr(smem);
-        for (int kb = 0; kb < KB && ok; ++kb) {
-            const int st = kb % kStages;
-            if (!wait_bar(&full[st], (kb / kStages) & 1, p, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t a = base + st * kStageBytes;
+        // (one lane chosen by elect.sync: a branch on the lane index costs the
+        // issuing thread more per tcgen05.mma than the product takes)
+        if (elect_one()) {
+            const uint32_t base = smem_addr(smem);
+            for (int kb = 0; kb < KB && ok; ++kb) {
+                const int st = kb % kStages;
+                if (!wait_bar(&full[st], (kb / kStages) & 1, p, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = base + st * kStageBytes;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = smem_desc_sw128(a + kk * 32, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(a + kTileBytes + kk * 32, 16, 1024);
-                mma_tf32_ss(tbase, ad, bd, kIdescTF32, (kb > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(a + kk * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(a + kTileBytes + kk * 32, 16, 1024);
+                    mma_tf32_ss(tbase, ad, bd, kIdescTF32, (kb > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&empty[st]);
             }
-            mma_commit(&empty[st]);
+            mma_commit(done);
+            mma_commit(drain);
+            drain_bar(drain, 0, p);
         }
-        mma_commit(done);
-        mma_commit(drain);
-        drain_bar(drain, 0, p);
     }
     __syncwarp();
 

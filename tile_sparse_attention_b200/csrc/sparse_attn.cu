@@ -19,7 +19,7 @@
 //                   p_t x p_h x p_w box of the token grid, fetched by a 5-D TMA
 //                   copy (d, Ws, Hs, T, B*H) with a 64-channel, 128-byte-swizzled
 //                   box, so no gather kernel or token permutation is needed;
-//       warp 1      allocates tensor memory; lane 0 issues every tcgen05.mma:
+//       warp 1      allocates tensor memory; one elected lane issues every tcgen05.mma:
 //                   S_j = Q K_j^T and O += P_j V_j, both with the A operand (Q,
 //                   P_j) read from tensor memory and B (K_j, V_j) from shared
 //                   memory, so shared memory only carries the K and V tiles (an

@@ -18,7 +18,7 @@
 //   * warp 0 (TMA producer) streams Q of each query tile into one staging
 //     buffer, and the selected K and V tiles of all its query tiles through
 //     one NS-deep ring (the key tiles of the CTA form one stream g = n*k + j);
-//   * warp 1 allocates tensor memory once; its lane 0 issues S_g = Q_n K_g^T
+//   * warp 1 allocates tensor memory once; one elected lane issues S_g = Q_n K_g^T
 //     (A = Q_n from one of two TMEM Q buffers, B = K from the ring) and
 //     O += P_g V_g, with S_{g+2} queued behind P_g V_g across tile boundaries;
 //   * warps 4..7 (thread = query row) run the online softmax of tile n, copy
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
+        if (elect_one()) {
             const uint32_t tS = tbase + C::kTmemS;
             const uint32_t tQ = tbase + C::kTmemQ;
             const uint32_t tO = tbase + C::kTmemO;

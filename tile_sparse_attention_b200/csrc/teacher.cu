@@ -18,7 +18,7 @@
 //
 // Kernel layout (one CTA per query tile, 256 threads): warp 0 streams Q once
 // and every K tile through an NS-deep TMA ring; warp 1 allocates tensor
-// memory and its lane 0 issues S_j = Q K_j^T (A = Q from tensor memory) into
+// memory and one elected lane issues S_j = Q K_j^T (A = Q from tensor memory) into
 // two TMEM S buffers; warps 4..7 (thread = query row) read S_j, take the row
 // max and fold the tile maximum into T.  All waits are bounded.
 #include "internal.h"
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
+        if (elect_one()) {
             const uint32_t k_addr = smem_addr(sK);
             const uint32_t tQ = tbase + C::kTmemQ;
             bool ok = wait_bar(bar_q_tmem, 0, p, abort_flag);
