@@ -97,7 +97,8 @@ veda_status encode_tile_map(CUtensorMap* map, const void* base, const Problem& p
 // dims (64, Ws, Hs, T*B*H, 2), box (64, p_w, p_h, p_t, 2) -> two 128-row planes.
 veda_status encode_tile_map_2c(CUtensorMap* map, const void* base, const Problem& pr,
                                const int* shape);
-veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows, int cols);
+veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows, int cols,
+                            int box_rows = 128);
 // Time limit of a device wait (VEDA_WAIT_LIMIT_MS, default 10 s).
 unsigned long long wait_limit_ns();
 

@@ -13,12 +13,18 @@
 // fp32 product by at most about 3 * 2^-21 |q||k| per term (the dropped lo*lo
 // term and the TF32 truncation of lo); accumulation is fp32 in tensor memory.
 // S = q^ k^^T is then one kind::tf32 GEMM with K = 9d:
-//   * one CTA per 128 x 128 block of S of one head; 128 threads;
-//   * warp 0 lane 0 streams 32-wide K blocks of q^ and k^ (128 rows x 128 B,
-//     128-byte swizzle) by TMA into a 3-stage ring;
-//   * warp 1 allocates 128 TMEM columns; one of its lanes, chosen by
-//     elect.sync, issues 4 tcgen05.mma (M = N = 128, K = 8) per K block;
+//   * one CTA per 128 x BN block of S of one head (BN = 256 for large score
+//     matrices: the operands come from L2 at about the rate TMA can move
+//     them, and a wider block loads each q^ row for twice the columns;
+//     BN = 128 when 256 would pad the columns by more than a tenth or leave
+//     fewer than two blocks per SM); 128 threads;
+//   * warp 0 lane 0 streams 32-wide K blocks of q^ (128 rows) and k^ (BN
+//     rows), 128 B per row with the 128-byte swizzle, by TMA into a ring;
+//   * warp 1 allocates BN TMEM columns; one of its lanes, chosen by
+//     elect.sync, issues 4 tcgen05.mma (M = 128, N = BN, K = 8) per K block;
 //   * all four warps read the accumulator back (thread = row) and store S.
+// Every S element accumulates the same products in the same order for
+// either BN, so the two block widths give identical S.
 // Waits are bounded (VEDA_ERR_TIMEOUT in the status word, then a bounded drain
 // of the copies and products in flight before tensor memory is freed; S is not
 // written by a CTA that gave up).
@@ -31,13 +37,18 @@ namespace veda {
 namespace {
 
 constexpr int kScoreThreads = 128;
-constexpr int kStages = 3;
-constexpr int kTileBytes = 128 * 128;             // 128 rows x 32 fp32
-constexpr int kStageBytes = 2 * kTileBytes;       // A and B
-constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
-// kind::tf32, fp32 accumulate, both operands K-major, M = N = 128
-constexpr uint32_t kIdescTF32 = (1u << 4) | (2u << 7) | (2u << 10) | ((128u >> 3) << 17) |
-                                ((128u >> 4) << 24);
+
+template <int BN>
+struct ScoreCfg {
+    static constexpr int kStages = BN == 256 ? 4 : 3;
+    static constexpr int kTileA = 128 * 128;  // 128 rows x 32 fp32
+    static constexpr int kTileB = BN * 128;   // BN rows x 32 fp32
+    static constexpr int kStageBytes = kTileA + kTileB;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
+    // kind::tf32, fp32 accumulate, both operands K-major, M = 128, N = BN
+    static constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) |
+                                       ((uint32_t)(BN >> 3) << 17) | ((128u >> 4) << 24);
+};
 
 struct __align__(64) ScoreParams {
     CUtensorMap mapA;  // q^: rows B*H*nT, K = 9d
@@ -49,8 +60,12 @@ struct __align__(64) ScoreParams {
     int withhold_fill;  // failure-detection test only: the first K block is never loaded
 };
 
+template <int BN>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_tc_kernel(const __grid_constant__ ScoreParams p) {
+    using C = ScoreCfg<BN>;
+    constexpr int kStages = C::kStages;
+    constexpr int kStageBytes = C::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -62,7 +77,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int j0 = blockIdx.x * 128, i0 = blockIdx.y * 128, bh = blockIdx.z;
+    const int j0 = blockIdx.x * BN, i0 = blockIdx.y * 128, bh = blockIdx.z;
     const int rowA = bh * p.nT + i0, rowB = bh * p.nT + j0;
     const int KB = p.kblocks;
 
@@ -77,7 +92,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 128);
+        tmem_alloc(tmem_slot, BN);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -103,7 +118,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             uint8_t* a = smem + st * kStageBytes;
             mbar_arrive_expect_tx(&full[st], kStageBytes);
             tma_load_2d(a, &p.mapA, &full[st], kb * 32, rowA);
-            tma_load_2d(a + kTileBytes, &p.mapB, &full[st], kb * 32, rowB);
+            tma_load_2d(a + C::kTileA, &p.mapB, &full[st], kb * 32, rowB);
             issued = kb + 1;
         }
         for (int st = 0; st < kStages; ++st)  // drain: the last fill of every stage
@@ -126,8 +141,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t ad = smem_desc_sw128(a + kk * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(a + kTileBytes + kk * 32, 16, 1024);
-                    mma_tf32_ss(tbase, ad, bd, kIdescTF32, (kb > 0 || kk > 0) ? 1u : 0u);
+                    const uint64_t bd = smem_desc_sw128(a + C::kTileA + kk * 32, 16, 1024);
+                    mma_tf32_ss(tbase, ad, bd, C::kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&empty[st]);
             }
@@ -152,7 +167,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         float* srow = p.S + ((size_t)bh * p.nT + i) * p.nT;
         const bool vec = (p.nT % 4) == 0;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < BN / 32; ++cc) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(taddr + cc * 32, v);
             tmem_wait_ld();
@@ -176,8 +191,22 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tbase, 128);
+        tmem_dealloc(tbase, BN);
     }
+}
+
+template <int BN>
+veda_status launch_score_bn(ScoreParams& prm, const Problem& pr, const float* kext, long long rows,
+                            int kx, cudaStream_t s) {
+    using C = ScoreCfg<BN>;
+    veda_status st;
+    if ((st = encode_rows_map(&prm.mapB, kext, rows, kx, BN)) != VEDA_OK) return st;
+    cudaError_t err = cudaFuncSetAttribute(score_tc_kernel<BN>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (err != cudaSuccess) return cuda_check(err, "score smem attribute");
+    dim3 grid((pr.nT + BN - 1) / BN, (pr.nT + 127) / 128, pr.B * pr.H);
+    score_tc_kernel<BN><<<grid, kScoreThreads, C::kSmemBytes, s>>>(prm);
+    return cuda_check(cudaGetLastError(), "score launch");
 }
 
 }  // namespace
@@ -190,7 +219,6 @@ veda_status launch_score(const Problem& pr, const float* qext, const float* kext
     const int kx = 9 * pr.d;
     veda_status st;
     if ((st = encode_rows_map(&prm.mapA, qext, rows, kx)) != VEDA_OK) return st;
-    if ((st = encode_rows_map(&prm.mapB, kext, rows, kx)) != VEDA_OK) return st;
     prm.S = S;
     prm.status = status;
     prm.nT = pr.nT;
@@ -198,13 +226,13 @@ veda_status launch_score(const Problem& pr, const float* qext, const float* kext
     prm.wait_limit_ns = wait_limit_ns();
     // Test hook for the bounded waits (nothing in normal use sets the variable).
     prm.withhold_fill = getenv("VEDA_TEST_WITHHOLD_ARRIVE") != nullptr ? 1 : 0;
-    cudaError_t err = cudaFuncSetAttribute(score_tc_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (err != cudaSuccess) return cuda_check(err, "score smem attribute");
-    const int tiles = (pr.nT + 127) / 128;
-    dim3 grid(tiles, tiles, pr.B * pr.H);
-    score_tc_kernel<<<grid, kScoreThreads, kSmemBytes, s>>>(prm);
-    return cuda_check(cudaGetLastError(), "score launch");
+    // 256-column blocks when they pad the columns by at most a tenth more than
+    // 128-column ones and still give every SM two blocks
+    const long long pad128 = (pr.nT + 127) / 128 * 128, pad256 = (pr.nT + 255) / 256 * 256;
+    const long long blocks256 = (pad256 / 256) * ((pr.nT + 127) / 128) * (long long)pr.B * pr.H;
+    if (pad256 * 10 <= pad128 * 11 && blocks256 >= 2LL * sm_count())
+        return launch_score_bn<256>(prm, pr, kext, rows, kx, s);
+    return launch_score_bn<128>(prm, pr, kext, rows, kx, s);
 }
 
 }  // namespace veda

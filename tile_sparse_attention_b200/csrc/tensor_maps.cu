@@ -76,12 +76,13 @@ veda_status encode_tile_map_2c(CUtensorMap* map, const void* base, const Problem
     return VEDA_OK;
 }
 
-veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows, int cols) {
+veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows, int cols,
+                            int box_rows) {
     EncodeTiledFn enc = get_encode_fn();
     if (enc == nullptr) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
-    const cuuint32_t box[2] = {32, 128};
+    const cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
