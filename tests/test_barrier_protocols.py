@@ -1,4 +1,6 @@
-"""Barrier protocols of the three attention kernels, checked by random interleaving.
+"""Barrier protocols of the three attention kernels and of the persistent score
+GEMM (score_tc.cu: a TMA ring running on across blocks of S, two tensor-memory
+accumulators drained by four epilogue warps), checked by random interleaving.
 
 The tile-skipping attention kernels (sparse_attn.cu: one CTA per query tile;
 sparse_attn_persistent.cu: persistent CTAs looping over query tiles with one
@@ -465,3 +467,85 @@ def test_a_planted_refill_race_is_caught():
         except AssertionError:
             caught += 1
     assert caught > 0
+
+
+# ------------------------------------------------------------------ score GEMM
+def model_score(n_blocks, KB, NS, seed, release_wait=True, acc_wait=True):
+    """score_tc.cu: a persistent CTA computes n_blocks blocks of S, each KB K
+    blocks long; the TMA ring of NS stages runs on across blocks; block lt is
+    accumulated in tensor-memory accumulator lt & 1, released by the four
+    epilogue warps once they have read it back."""
+    rnd = random.Random(seed)
+    full = [Bar(1) for _ in range(NS)]
+    empty = [Bar(1) for _ in range(NS)]
+    acc_full, acc_empty = [Bar(1), Bar(1)], [Bar(4), Bar(4)]
+    tma, tc = [], []
+    st = {"ring": [None] * NS, "acc": [None, None]}  # acc: (block, products so far)
+    written = []
+
+    def producer():
+        g = 0
+        for lt in range(n_blocks):
+            for kb in range(KB):
+                s, n = g % NS, g // NS
+                if n > 0 and release_wait:
+                    yield lambda s=s, n=n: passed(empty[s], n - 1)
+
+                def landed(s=s, lt=lt, kb=kb):
+                    st["ring"][s] = (lt, kb)
+                    full[s].arrive()
+                tma.append(landed)
+                g += 1
+
+    def issuer():
+        g = 0
+        for lt in range(n_blocks):
+            a, use = lt & 1, lt >> 1
+            if use > 0 and acc_wait:
+                yield lambda a=a, use=use: passed(acc_empty[a], use - 1)
+            for kb in range(KB):
+                s = g % NS
+                yield lambda s=s, g=g: passed(full[s], g // NS)
+
+                def mma(s=s, lt=lt, kb=kb, a=a):
+                    assert st["ring"][s] == (lt, kb), "product reads the wrong ring stage"
+                    if kb == 0:
+                        st["acc"][a] = (lt, 1)
+                    else:
+                        assert st["acc"][a] == (lt, kb), "accumulator overwritten mid-block"
+                        st["acc"][a] = (lt, kb + 1)
+                tc.append(mma)
+                tc.append(lambda s=s: empty[s].arrive())
+                g += 1
+            tc.append(lambda a=a: acc_full[a].arrive())
+
+    def epilogue(w):
+        for lt in range(n_blocks):
+            a, use = lt & 1, lt >> 1
+            yield lambda a=a, use=use: passed(acc_full[a], use)
+            assert st["acc"][a] == (lt, KB), "epilogue reads an incomplete block"
+            yield lambda: True  # the read takes time: other roles may move
+            assert st["acc"][a] == (lt, KB), "accumulator overwritten while being read"
+            written.append((w, lt))
+            acc_empty[a].arrive()
+
+    run([producer(), issuer()] + [epilogue(w) for w in range(4)], tma, tc, rnd)
+    assert sorted(written) == [(w, lt) for w in range(4) for lt in range(n_blocks)]
+
+
+@pytest.mark.parametrize("n_blocks,KB,NS", [(1, 3, 4), (2, 1, 4), (5, 3, 4), (7, 2, 6), (4, 9, 4),
+                                            (6, 1, 2)])
+def test_score_protocol(n_blocks, KB, NS):
+    for seed in range(300):
+        model_score(n_blocks, KB, NS, seed)
+
+
+@pytest.mark.parametrize("mistake", ["release_wait", "acc_wait"])
+def test_score_planted_mistakes_are_caught(mistake):
+    caught = 0
+    for seed in range(300):
+        try:
+            model_score(5, 3, 4, seed, **{mistake: False})
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"dropping {mistake} went unnoticed"
