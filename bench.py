@@ -745,12 +745,16 @@ def main():
                     help="time the attention alone on estimator, random and local index lists")
     ap.add_argument("--rows", default="",
                     help="comma list of f1,f2,f3,f4: time the next rows instead")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="long_video with its first N heads only (a smaller case for counter captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "veda":
         args.warmup = 3
     if args.workload.startswith("sweep:"):
         _, T, s = args.workload.split(":")
         w = workloads.sweep(int(T), int(s))
+    elif args.heads and args.workload == "long_video":
+        w = workloads.long_video(H=args.heads)
     else:
         w = workloads.CONFIGS[args.workload]()
     if args.sweep:

@@ -84,7 +84,10 @@ def test_topk_bit_exact_on_extreme_rows(vb, oracle):
     spacing, coarse quantisation (hundreds of equal scores at the threshold), and
     k = nT.  The selection must still equal the oracle's exactly."""
     rng = np.random.default_rng(11)
-    for nT, k in ((1920, 96), (600, 30), (37, 5), (300, 300), (4097, 200)):
+    # register kernel: 1920, 600, 37, 300, 1001 (rows not 16-byte aligned), 1540
+    # (padded float4 groups); shared-memory kernel: 1999 (unaligned), 4097
+    for nT, k in ((1920, 96), (600, 30), (37, 5), (300, 300), (1001, 50), (1540, 77),
+                  (1999, 100), (4097, 200)):
         H = 8
         w = workloads.custom("topk_x", 1, H, 64, (1, 1, 64 * nT), [(1, 1, 64)], k)
         S = rng.standard_normal((1, H, nT, nT)).astype(np.float32)

@@ -139,7 +139,8 @@ def test_selection_matches_stable_sort_on_stress_rows():
 
 
 # ---------------------------------------------------------------- rows of up to 2048 scores
-# topk.cu keeps such a row in registers: lane l holds the groups of four scores
+# (up to 1024 when a row does not start on a 16-byte boundary) topk.cu keeps
+# such a row in registers: lane l holds the groups of four scores
 # l, l + 32, ... (G = ceil(nT / 128) per lane, padding read as NaN), buckets are
 # 7-bit, floor(127 * sat(fl(fl(x - min) * fl(1 / range)))) with NaN sent to 0 by
 # the saturation, packed four per 32-bit word as 0x80 | bucket; byte-parallel

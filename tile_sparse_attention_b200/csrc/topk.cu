@@ -665,10 +665,14 @@ veda_status launch_topk_reg_g(const TopkParams& prm, int g, cudaStream_t s) {
     if (g <= 2) return launch_topk_reg<2, ALIGNED>(prm, s);
     if (g <= 4) return launch_topk_reg<4, ALIGNED>(prm, s);
     if (g <= 5) return launch_topk_reg<5, ALIGNED>(prm, s);
-    if (g <= 8) return launch_topk_reg<8, ALIGNED>(prm, s);
-    if (g <= 12) return launch_topk_reg<12, ALIGNED>(prm, s);
-    if (g <= 15) return launch_topk_reg<15, ALIGNED>(prm, s);
-    return launch_topk_reg<16, ALIGNED>(prm, s);
+    if constexpr (!ALIGNED) {
+        return launch_topk_reg<8, ALIGNED>(prm, s);  // rows of up to 1024 scores
+    } else {
+        if (g <= 8) return launch_topk_reg<8, ALIGNED>(prm, s);
+        if (g <= 12) return launch_topk_reg<12, ALIGNED>(prm, s);
+        if (g <= 15) return launch_topk_reg<15, ALIGNED>(prm, s);
+        return launch_topk_reg<16, ALIGNED>(prm, s);
+    }
 }
 
 template <int W, int LOADS>
@@ -693,14 +697,15 @@ veda_status launch_topk(const Problem& pr, const float* S, uint8_t* mask, int32_
     prm.rows = (long long)pr.B * pr.H * pr.nT;
     prm.nT = pr.nT;
     prm.k = pr.k;
-    // rows of up to 2048 scores: in registers, 128 scores per float4 group of
-    // every lane; longer rows: in shared memory, four warps (rows) per block
-    // up to 4096 tiles (<= 74 KB), one above (<= 66 KB at the 16384-tile limit)
-    if (pr.nT <= 128 * kRegMaxG) {
-        const int g = (pr.nT + 127) / 128;
-        return (pr.nT & 3) == 0 ? launch_topk_reg_g<true>(prm, g, s)
-                                : launch_topk_reg_g<false>(prm, g, s);
-    }
+    // rows of up to 2048 scores (1024 when they do not start on 16-byte
+    // boundaries: their single-score loads need more registers): in registers,
+    // 128 scores per float4 group of every lane; longer rows: in shared
+    // memory, four warps (rows) per block up to 4096 tiles (<= 74 KB), one
+    // above (<= 66 KB at the 16384-tile limit)
+    if ((pr.nT & 3) == 0 && pr.nT <= 128 * kRegMaxG)
+        return launch_topk_reg_g<true>(prm, (pr.nT + 127) / 128, s);
+    if ((pr.nT & 3) != 0 && pr.nT <= 1024)
+        return launch_topk_reg_g<false>(prm, (pr.nT + 127) / 128, s);
     if (pr.nT <= 4096) return launch_topk_w<4, 16>(prm, s);
     return launch_topk_w<1, 16>(prm, s);
 }
