@@ -291,6 +291,21 @@ def test_forward_long_video(vb, oracle):
     _forward_parity(vb, oracle, w, list(range(w.H)), 16)
 
 
+def test_forward_batch2_mixed_tile_shapes(vb, oracle):
+    """B = 2 with four head-aware tile shapes (32 tiles, k = 7): the mask prep
+    and every query tile's attention of every (b, h) against the oracle."""
+    w = workloads.custom("b2mix", 2, 4, 128, (8, 16, 32),
+                         [(1, 8, 16), (2, 8, 8), (4, 4, 8), (2, 8, 8)], 7)
+    _forward_parity(vb, oracle, w, list(range(w.H)), w.nT)
+
+
+def test_forward_batch2_wide_score_blocks(vb, oracle):
+    """B = 2, H = 6, 1,024 tiles, k = 51: enough 128 x 256 blocks of S that the
+    score GEMM takes its 256-column blocks, walked across both batch entries."""
+    w = workloads.custom("b2wide", 2, 6, 128, (16, 64, 128), [(2, 8, 8)], 51)
+    _forward_parity(vb, oracle, w, list(range(w.H)), 4)
+
+
 @pytest.mark.parametrize("T", workloads.SWEEP_T)
 @pytest.mark.parametrize("s", workloads.SWEEP_SPARSITY)
 def test_forward_sweep_points(vb, oracle, T, s):
