@@ -346,11 +346,13 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
-// Rows of up to 2048 scores: the row stays in registers.
+// Rows of up to 2048 scores (1024 for rows that do not start on a 16-byte
+// boundary): the row stays in registers.
 //
 // Lane l holds the float4 groups l, l + 32, ... (G of them), and the next row
-// is loaded into the same registers once the current one's bucket b* scores
-// have been gathered, so its loads land while this row's selection finishes.  The scores become 7-bit buckets,
+// is loaded into the same registers once the current one's bucket-b* scores
+// have been gathered, so its loads land while this row's selection finishes.
+// The scores become 7-bit buckets,
 //   bucket(x) = floor(127 * sat(fl(fl(x - min) * inv))),  inv = 1 / (max - min),
 // a non-decreasing function of x in which equal scores (-0.0 and +0.0
 // included) share a bucket; `sat` clamps to [0, 1] and sends NaN to 0, so the
@@ -362,13 +364,14 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(const __grid_constant_
 //      reduced over the warp, gives the bucket b* of the k-th largest score and
 //      the number of scores above it;
 //   2. the scores of bucket b* (a handful for smooth rows) are gathered from
-//      the registers and their exact threshold found as in the kernel above (pairwise ranks for up to 32,
-//      an 8-bit radix select otherwise, or over the whole row if more than
-//      kCandCap share the bucket); the chosen ones of b* are marked in a bitmap;
+//      the registers and their exact threshold found as in the kernel above
+//      (pairwise ranks for up to 32, an 8-bit radix select otherwise, or over
+//      the whole row, re-read, if more than kCandCap share the bucket); the
+//      chosen ones of b* are marked in a bitmap;
 //   3. the selected bytes of every packed word (buckets above b*, plus the
 //      bitmap) give per-lane counts, whose prefix over the warp comes from four
-//      counts per 32-bit word in one scan, and the index list is written already
-//      ascending.
+//      counts per 32-bit word in one scan, and the index list is written
+//      already ascending.
 
 constexpr int kRegWarps = 4;
 constexpr int kRegMaxG = 16;                 // rows of up to 128 * 16 = 2048 scores
@@ -465,14 +468,16 @@ __global__ void __launch_bounds__(kRegWarps * 32, G >= 12 ? 4 : G >= 5 ? 5 : 6)
         }
         // a zero or non-finite range puts every score in bucket 0 (still exact)
         const float range = __fsub_rn(mx, mn);
-        const float inv = (range > 0.f && range <= FLT_MAX) ? fminf(__frcp_rn(range), FLT_MAX) : 0.f;
+        const float inv =
+            (range > 0.f && range <= FLT_MAX) ? fminf(__frcp_rn(range), FLT_MAX) : 0.f;
         uint32_t pk[G];
 #pragma unroll
         for (int u = 0; u < G; ++u) pk[u] = pack_buckets(v[u], mn, inv);
         for (int w = lane; w < kRegBitmapWords; w += 32) bm[w] = 0u;
         if (lane == 0) *ncand = 0u;
 
-        // ---- 1. bucket b* of the k-th largest score: count(bucket >= lo) >= k > count(bucket >= hi)
+        // ---- 1. bucket b* of the k-th largest score:
+        //      count(bucket >= lo) >= k > count(bucket >= hi)
         uint32_t lo = 0, hi = 128, above = 0;
 #pragma unroll 1
         for (int it = 0; it < 7; ++it) {
@@ -506,7 +511,8 @@ __global__ void __launch_bounds__(kRegWarps * 32, G >= 12 ? 4 : G >= 5 ? 5 : 6)
                     const int e = (__ffs(eq) - 8) >> 3;
                     eq &= eq - 1u;
                     if (j0 + e < nT) {
-                        const float x = e == 0 ? v[u].x : e == 1 ? v[u].y : e == 2 ? v[u].z : v[u].w;
+                        const float x =
+                            e == 0 ? v[u].x : e == 1 ? v[u].y : e == 2 ? v[u].z : v[u].w;
                         const uint32_t pos = atomicAdd(ncand, 1u);
                         if (pos < (uint32_t)kCandCap) {
                             ck[pos] = order_key(x);
@@ -521,7 +527,8 @@ __global__ void __launch_bounds__(kRegWarps * 32, G >= 12 ? 4 : G >= 5 ? 5 : 6)
             const long long nrow = row + stride;
             if (nrow < p.rows) {
 #pragma unroll
-                for (int u = 0; u < G; ++u) v[u] = load_group<ALIGNED>(p.S + nrow * nT, 32 * u + lane, nT);
+                for (int u = 0; u < G; ++u)
+                    v[u] = load_group<ALIGNED>(p.S + nrow * nT, 32 * u + lane, nT);
             }
         }
         __syncwarp();
@@ -593,7 +600,8 @@ __global__ void __launch_bounds__(kRegWarps * 32, G >= 12 ? 4 : G >= 5 ? 5 : 6)
         for (int u = 0; u < G; ++u) {
             const int g = 32 * u + lane;
             const uint32_t nib = (bm[g >> 3] >> (4 * (g & 7))) & 0xfu;  // chosen scores of b*
-            const uint32_t m = ((pk[u] - T) & 0x80808080u) | (((nib * 0x00204081u) & 0x01010101u) << 7);
+            const uint32_t m =
+                ((pk[u] - T) & 0x80808080u) | (((nib * 0x00204081u) & 0x01010101u) << 7);
             pk[u] = m;
             sw[u >> 2] |= (uint32_t)__popc(m) << (8 * (u & 3));
         }
