@@ -47,10 +47,13 @@ veda_status launch_check_index(const int32_t* idx, long long rows, int k, int nT
 // error after checking the launch.
 veda_status launch_tripool(const Problem& pr, const uint16_t* Q, const uint16_t* K, float* statsQ,
                            float* statsK, cudaStream_t s);
-// Projection of statsQ (side 0) or statsK (side 1) into the TF32-split score
-// operand layout [B*H*nT][9d] (see tile_score.cu).
-veda_status launch_project(const Problem& pr, const float* stats, const float* W, float* out,
-                           int side, cudaStream_t s);
+// Both projections in one launch on the tensor cores (proj_tc.cu): statsQ . Wq
+// into qt and statsK . Wk into kt, in the TF32-split score operand layout
+// [B*H*nT][9d] (query side [hi|hi|lo], key side [hi|lo|hi] per statistic);
+// status: device status word.
+veda_status launch_project_pair(const Problem& pr, const float* statsQ, const float* statsK,
+                                const float* Wq, const float* Wk, float* qt, float* kt,
+                                int* status, cudaStream_t s);
 // S = q^ k^^T on the tensor cores (score_tc.cu); status: device status word.
 veda_status launch_score(const Problem& pr, const float* qext, const float* kext, float* S,
                          int* status, cudaStream_t s);
@@ -102,7 +105,7 @@ veda_status encode_rows_map(CUtensorMap* map, const float* base, long long rows,
 // Time limit of a device wait (VEDA_WAIT_LIMIT_MS, default 10 s).
 unsigned long long wait_limit_ns();
 
-// Batched fp32 SIMT GEMM (tile_score.cu): C[z] (+)= op(A[z']) . op(B[z''])
+// Batched fp32 SIMT GEMM (sgemm.cu): C[z] (+)= op(A[z']) . op(B[z''])
 // with z' = z % a_batch_mod, z'' = z % b_batch_mod (when > 0); a_t: A stored
 // K x M; b_t: B stored N x K.  K must be a multiple of 8.
 veda_status launch_sgemm(const float* A, const float* B, float* C, int M, int N, int K, int lda,

@@ -95,9 +95,9 @@ veda_status veda_tile_score_noalloc(const veda_problem* p, const float* statsQ,
     float* kt = reinterpret_cast<float*>(base + VEDA_STATUS_BYTES + stats);
     if ((st = veda::cuda_check(cudaMemsetAsync(base, 0, VEDA_STATUS_BYTES, s), "status reset")))
         return st;
-    if ((st = veda::launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
-    if ((st = veda::launch_project(pr, statsK, Wk, kt, 1, s))) return st;
-    return veda::launch_score(pr, qt, kt, S, reinterpret_cast<int*>(base), s);
+    int* status = reinterpret_cast<int*>(base);
+    if ((st = veda::launch_project_pair(pr, statsQ, statsK, Wq, Wk, qt, kt, status, s))) return st;
+    return veda::launch_score(pr, qt, kt, S, status, s);
 }
 
 veda_status veda_noalloc_get_status(veda_stream_t stream, int32_t* device_status) {

@@ -1,20 +1,11 @@
-// tile_score.cu -- head-specific projection of the TripPool statistics and the
-// tile-pair score matrix.
-//
-// "Veda: Scalable Video Diffusion via Distilled Sparse Attention" (project
-// page), "Attention Structure Distillation", Estimator: head-specific Q/K
-// projections reconstruct the dense tile distribution from the average,
-// maximum and minimum statistics; "Theoretical Rationale" 4: the estimator
-// yields a score for every key tile before Top-k.
-//
-//   projection: q~[b,h] (3nT x d) = statsQ[b,h] (3nT x d) . Wq[h] (d x d)
-//
-// A small fp32 contraction on the FP32 SIMT pipes: a batched register-blocked
-// SGEMM, 128 x 128 block tile, 8 x 8 outputs per thread, double-buffered
-// shared memory.  Its epilogue writes each projected value x as the TF32 pair
-// hi = x rounded to TF32, lo = x - hi, laid out per tile as
-//   query side [hi | hi | lo],  key side [hi | lo | hi]   (each 3d long),
-// which is the operand layout of the tensor-core score GEMM (score_tc.cu).
+// sgemm.cu -- batched register-blocked fp32 SIMT GEMM for the distillation
+// products ("Principle 01 Full-Attention Structure Distillation" and
+// "Theoretical Rationale" 4 of the Veda project page: the loss gradients
+// dL/dW_q and dL/dW_k are fp32 matrix products of the statistics and the
+// score gradient).  128 x 128 block tile, 8 x 8 outputs per thread,
+// double-buffered shared memory; transposed-A, transposed-B and accumulate
+// modes.  (The estimator's forward projection runs on the tensor cores in
+// proj_tc.cu.)
 #include "internal.h"
 
 namespace veda {
@@ -31,17 +22,9 @@ struct GemmParams {
     int lda, ldb, ldc;
     long long strideA, strideB, strideC;  // per batch entry
     int b_batch_mod;                      // >0: B index = batch % b_batch_mod
-    int split;                            // 0: plain C; 1: query-side split; 2: key-side split
-    int d;                                // head dimension (split layouts)
-    int accumulate;                       // plain C only: C += A . B
+    int accumulate;                       // C += A . B
     int a_batch_mod;                      // >0: A index = batch % a_batch_mod
 };
-
-// x = hi + lo with hi = x rounded to nearest TF32 (10 explicit mantissa bits)
-// and lo = x - hi (exact in fp32).
-__device__ __forceinline__ float tf32_hi(float x) {
-    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
-}
 
 // C[z] = A[z] . B[z]  (B_T = false: B is K x N row-major)
 // C[z] = A[z] . B[z]^T (B_T = true: B is N x K row-major)
@@ -154,20 +137,6 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const __grid_constant__ Gemm
         for (int half = 0; half < 2; ++half) {
             const int n = n0 + half * 64 + tx * 4;
             const float* v = &acc[i][half * 4];
-            if (p.split != 0) {
-                // row m = 3 j + s of the projection -> tile j, positions s*d + n
-                // of the three 3d-long segments; N = d is a multiple of 64
-                if (n >= p.N) continue;
-                const int d = p.d, j = m / 3, srow = m % 3;
-                float* row = C + (long long)j * 9 * d + srow * d + n;
-                float4 hi, lo;
-                hi.x = tf32_hi(v[0]); hi.y = tf32_hi(v[1]); hi.z = tf32_hi(v[2]); hi.w = tf32_hi(v[3]);
-                lo = make_float4(v[0] - hi.x, v[1] - hi.y, v[2] - hi.z, v[3] - hi.w);
-                *reinterpret_cast<float4*>(row) = hi;
-                *reinterpret_cast<float4*>(row + 3 * d) = (p.split == 1) ? hi : lo;
-                *reinterpret_cast<float4*>(row + 6 * d) = (p.split == 1) ? lo : hi;
-                continue;
-            }
             float* dst = C + (long long)m * p.ldc + n;
             if (vec && n + 3 < p.N) {
                 float4 o = make_float4(v[0], v[1], v[2], v[3]);
@@ -185,29 +154,6 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const __grid_constant__ Gemm
 }
 
 }  // namespace
-
-veda_status launch_project(const Problem& pr, const float* stats, const float* W, float* out,
-                           int side, cudaStream_t s) {
-    GemmParams g{};
-    g.A = stats;
-    g.B = W;
-    g.C = out;
-    g.M = 3 * pr.nT;
-    g.N = pr.d;
-    g.K = pr.d;
-    g.lda = pr.d;
-    g.ldb = pr.d;
-    g.ldc = 9 * pr.d;
-    g.strideA = (long long)3 * pr.nT * pr.d;
-    g.strideB = (long long)pr.d * pr.d;
-    g.strideC = (long long)9 * pr.nT * pr.d;
-    g.b_batch_mod = pr.H;
-    g.split = side == 0 ? 1 : 2;
-    g.d = pr.d;
-    dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM, pr.B * pr.H);
-    sgemm_kernel<false><<<grid, 256, 0, s>>>(g);
-    return cuda_check(cudaGetLastError(), "projection launch");
-}
 
 veda_status launch_sgemm(const float* A, const float* B, float* C, int M, int N, int K, int lda,
                          int ldb, int ldc, long long strideA, long long strideB, long long strideC,

@@ -147,8 +147,7 @@ veda_status forward_impl(const Problem& pr, const uint16_t* Q, const uint16_t* K
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
     veda_status st;
     if ((st = launch_tripool(pr, Q, K, statsQ, statsK, s))) return st;
-    if ((st = launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
-    if ((st = launch_project(pr, statsK, Wk, kt, 1, s))) return st;
+    if ((st = launch_project_pair(pr, statsQ, statsK, Wq, Wk, qt, kt, status, s))) return st;
     if ((st = launch_score(pr, qt, kt, S, status, s))) return st;
     if ((st = launch_topk(pr, S, mask_out, idx, s))) return st;
     return launch_sparse_attn(pr, Q, K, V, idx, pr.k, O, lse, status, s);
@@ -201,9 +200,9 @@ veda_status veda_tile_score(const veda_problem* p, const float* statsQ, const fl
     float* kt = reinterpret_cast<float*>(base + w.kt);
     if ((st = cuda_check(cudaMemsetAsync(base + w.status, 0, sizeof(int), s), "status reset")))
         return st;
-    if ((st = launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
-    if ((st = launch_project(pr, statsK, Wk, kt, 1, s))) return st;
-    return launch_score(pr, qt, kt, S, reinterpret_cast<int*>(base + w.status), s);
+    int* status = reinterpret_cast<int*>(base + w.status);
+    if ((st = launch_project_pair(pr, statsQ, statsK, Wq, Wk, qt, kt, status, s))) return st;
+    return launch_score(pr, qt, kt, S, status, s);
 }
 
 veda_status veda_topk_mask(const veda_problem* p, const float* S, uint8_t* mask, int32_t* idx,
@@ -256,8 +255,7 @@ veda_status veda_mask_fused(const veda_problem* p, const float* statsQ, const fl
     float* kt = reinterpret_cast<float*>(base + w.kt);
     int* status = reinterpret_cast<int*>(base + w.status);
     if ((st = cuda_check(cudaMemsetAsync(status, 0, sizeof(int), s), "status reset"))) return st;
-    if ((st = launch_project(pr, statsQ, Wq, qt, 0, s))) return st;
-    if ((st = launch_project(pr, statsK, Wk, kt, 1, s))) return st;
+    if ((st = launch_project_pair(pr, statsQ, statsK, Wq, Wk, qt, kt, status, s))) return st;
     return launch_score_topk(pr, qt, kt, mask, idx, status, s);
 }
 
