@@ -1,6 +1,8 @@
-"""Barrier protocols of the three attention kernels and of the persistent score
+"""Barrier protocols of the three attention kernels, of the persistent score
 GEMM (score_tc.cu: a TMA ring running on across blocks of S, two tensor-memory
-accumulators drained by four epilogue warps), checked by random interleaving.
+accumulators drained by four epilogue warps) and of the projection
+(proj_tc.cu: two raw buffers filled one half ahead, a shared lo buffer, two
+accumulators), checked by random interleaving.
 
 The tile-skipping attention kernels (sparse_attn.cu: one CTA per query tile;
 sparse_attn_persistent.cu: persistent CTAs looping over query tiles with one
@@ -546,6 +548,90 @@ def test_score_planted_mistakes_are_caught(mistake):
     for seed in range(300):
         try:
             model_score(5, 3, 4, seed, **{mistake: False})
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"dropping {mistake} went unnoticed"
+
+
+# ------------------------------------------------------------------ projection
+def model_projection(n_blocks, halves, seed, acc_wait=True, done_wait=True, full_wait=True):
+    """proj_tc.cu: warps 0..3 (one role: they act together) take each half of
+    a block's statistics from one of two raw buffers (the next half's copy goes
+    out once this half's products are issued), split it into a shared lo
+    buffer, and issue its products into accumulator lb & 1; warps 4..7 read a
+    finished accumulator back and release it."""
+    rnd = random.Random(seed)
+    full, done = Bar(1), Bar(1)
+    acc_full, acc_empty = [Bar(1), Bar(1)], [Bar(4), Bar(4)]
+    tma, tc = [], []
+    st = {"raw": [None, None], "lo": None, "acc": [None, None]}
+    written = []
+
+    def load(lb, hk, g):
+        def landed():
+            st["raw"][g & 1] = (lb, hk)
+            full.arrive()
+        tma.append(landed)
+
+    def main():
+        g = 0
+        if n_blocks:
+            load(0, 0, 0)
+        for lb in range(n_blocks):
+            a, use = lb & 1, lb >> 1
+            if use > 0 and acc_wait:
+                yield lambda a=a, use=use: passed(acc_empty[a], use - 1)
+            for hk in range(halves):
+                if full_wait:
+                    yield lambda g=g: passed(full, g)
+                st["lo"] = st["raw"][g & 1]  # the split reads the raw half, writes lo
+
+                def mma(lb=lb, hk=hk, g=g, a=a):
+                    assert st["raw"][g & 1] == (lb, hk), "products read the wrong raw half"
+                    assert st["lo"] == (lb, hk), "products read the wrong lo half"
+                    if hk == 0:
+                        st["acc"][a] = (lb, 1)
+                    else:
+                        assert st["acc"][a] == (lb, hk), "accumulator overwritten mid-block"
+                        st["acc"][a] = (lb, hk + 1)
+                tc.append(mma)
+                tc.append(done.arrive)
+                if hk + 1 == halves:
+                    tc.append(lambda a=a: acc_full[a].arrive())
+                if hk + 1 < halves:
+                    load(lb, hk + 1, g + 1)
+                elif lb + 1 < n_blocks:
+                    load(lb + 1, 0, g + 1)
+                if done_wait:
+                    yield lambda g=g: passed(done, g)
+                g += 1
+
+    def epilogue(w):
+        for lb in range(n_blocks):
+            a, use = lb & 1, lb >> 1
+            yield lambda a=a, use=use: passed(acc_full[a], use)
+            assert st["acc"][a] == (lb, halves), "epilogue reads an incomplete block"
+            yield lambda: True
+            assert st["acc"][a] == (lb, halves), "accumulator overwritten while being read"
+            written.append((w, lb))
+            acc_empty[a].arrive()
+
+    run([main()] + [epilogue(w) for w in range(4)], tma, tc, rnd)
+    assert sorted(written) == [(w, lb) for w in range(4) for lb in range(n_blocks)]
+
+
+@pytest.mark.parametrize("n_blocks,halves", [(1, 2), (2, 1), (5, 2), (7, 1), (4, 2)])
+def test_projection_protocol(n_blocks, halves):
+    for seed in range(300):
+        model_projection(n_blocks, halves, seed)
+
+
+@pytest.mark.parametrize("mistake", ["acc_wait", "done_wait", "full_wait"])
+def test_projection_planted_mistakes_are_caught(mistake):
+    caught = 0
+    for seed in range(300):
+        try:
+            model_projection(5, 2, seed, **{mistake: False})
         except AssertionError:
             caught += 1
     assert caught > 0, f"dropping {mistake} went unnoticed"

@@ -194,7 +194,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++lt) {
             const int acc = lt & 1, use = lt >> 1;
             // after an abort an accumulator may be incomplete: no more blocks are written
-            if (!warp_wait_bar(&acc_full[acc], use & 1, p, abort_flag) || *abort_flag) break;
+            if (!warp_wait_bar(&acc_full[acc], use & 1, p, abort_flag) ||
+                __any_sync(0xffffffffu, *abort_flag != 0))
+                break;  // the whole warp leaves: the tensor-memory loads below are warp-wide
             tc_fence_after();
             const int jb = t % p.tiles_j, rest = t / p.tiles_j;
             const int ib = rest % p.tiles_i, bh = rest / p.tiles_i;
