@@ -106,7 +106,7 @@ veda_status veda_tripool(const veda_problem* p, const uint16_t* Q, const uint16_
  *   ws    : device workspace of at least
  *           VEDA_STATUS_BYTES + 2 * B*H*nT*9*d*4 bytes (projected statistics,
  *           stored as TF32 hi/lo splits).
- * The projection is fp32; the score is a tensor-core product of three TF32
+ * The projection and the score are each a tensor-core product of three TF32
  * terms (hi.hi + hi.lo + lo.hi, fp32 accumulation), within about 3 * 2^-21 of
  * the fp32 product per term.
  */
