@@ -5,10 +5,12 @@ Parity rules (tolerances derived from the arithmetic):
 * TripPool max/min: bit-exact (a max of bf16 values is exact in fp32);
   avg: |gpu - oracle| <= (Bt - 1) * 2^-24 * mean|x| + 2^-24 * |avg|, the error
   bound of an fp32 sum of Bt terms followed by an exact division by 2^m.
-* scores: |gpu - oracle| <= 8e-5 * (|stats_q| |W_q|) . (|stats_k| |W_k|)^T: the
-  fp32 projection (d terms), the three-term TF32 product (<= 3 * 2^-21 per term)
-  and fp32 accumulation of 9d products: (d + 9d + 4) * 2^-24 + 3 * 2^-21 <= 7.8e-5
-  on the absolute terms.
+* scores: |gpu - oracle| <= 9e-5 * (|stats_q| |W_q|) . (|stats_k| |W_k|)^T: each
+  of the two projections is a three-term TF32 product with fp32 accumulation
+  of d terms (d * 2^-24 + 3 * 2^-21 relative to the absolute terms), the score
+  a three-term TF32 product (3 * 2^-21) accumulated over 9d terms in fp32:
+  (2d + 9d + 4) * 2^-24 + 9 * 2^-21 = 8.84e-5 at d = 128, worst case on the
+  absolute terms.
 * mask rows: bit-exact wherever the oracle's k-th and (k+1)-th scores differ
   by more than 1e-3 relative; in other rows the GPU row must hold exactly k
   tiles and every tile whose oracle score clears s_(k) by that margin.
@@ -27,7 +29,7 @@ from oracle import Oracle
 O_MAX_ABS = 2e-2
 O_MEAN_ABS = 5e-3
 LSE_ABS = 2e-3
-SCORE_GAMMA = 8e-5
+SCORE_GAMMA = 9e-5
 GAP_REL = 1e-3
 
 
